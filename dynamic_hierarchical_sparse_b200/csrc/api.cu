@@ -1,0 +1,320 @@
+// C ABI of libdhsa.so: argument validation, workspace carving and launches.
+// Every entry point returns a dhsa_status; nothing throws across the ABI.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/dhsa.h"
+#include "common.cuh"
+#include "launchers.h"
+
+namespace dhsa {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+constexpr int kMaxSelectCandidates = 12000;  // per-row staging in shared memory
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t budget_of(int i_local, const dhsa_budget& b) {
+  if (b.kind == DHSA_BUDGET_TOPK) return i_local < b.k ? i_local : b.k;
+  const int64_t want = (static_cast<int64_t>(i_local) * b.num + b.den - 1) / b.den;
+  return want < i_local ? want : i_local;
+}
+
+dhsa_status check_budget(const dhsa_budget& b) {
+  if (b.kind == DHSA_BUDGET_TOPK) return b.k >= 0 ? DHSA_OK : DHSA_ERR_INVALID_ARG;
+  if (b.kind == DHSA_BUDGET_FRACTION) return (b.num >= 0 && b.den >= 1) ? DHSA_OK : DHSA_ERR_INVALID_ARG;
+  return DHSA_ERR_INVALID_ARG;
+}
+
+dhsa_status check_problem(const dhsa_problem* p) {
+  if (p == nullptr) return DHSA_ERR_INVALID_ARG;
+  if (p->dtype != DHSA_BF16 && p->dtype != DHSA_F32) return DHSA_ERR_INVALID_ARG;
+  if (p->num_seqs < 0 || p->total_tokens < 0 || p->num_chunks < 0) return DHSA_ERR_INVALID_ARG;
+  if (p->num_q_heads < 1 || p->num_kv_heads < 1 || p->num_q_heads % p->num_kv_heads != 0)
+    return DHSA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) {
+    return p->head_dim > 0 ? DHSA_ERR_UNSUPPORTED : DHSA_ERR_INVALID_ARG;
+  }
+  if (p->num_chunks > 65535 || p->num_q_heads > 65535) return DHSA_ERR_UNSUPPORTED;
+  if (p->h_cu_seqlens == nullptr || p->h_chunk_bounds == nullptr || p->h_seq_chunk_ptr == nullptr)
+    return DHSA_ERR_INVALID_ARG;
+  if (p->cu_seqlens == nullptr || p->chunk_bounds == nullptr || p->seq_chunk_ptr == nullptr)
+    return DHSA_ERR_INVALID_ARG;
+  const int B = p->num_seqs, n = p->num_chunks;
+  const int32_t* cu = p->h_cu_seqlens;
+  const int32_t* bd = p->h_chunk_bounds;
+  const int32_t* sp = p->h_seq_chunk_ptr;
+  if (cu[0] != 0 || cu[B] != p->total_tokens) return DHSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (cu[b + 1] < cu[b]) return DHSA_ERR_INVALID_ARG;
+  if (bd[0] != 0 || bd[n] != p->total_tokens) return DHSA_ERR_INVALID_ARG;
+  for (int c = 0; c < n; ++c)
+    if (bd[c + 1] <= bd[c]) return DHSA_ERR_INVALID_ARG;  // chunks are non-empty
+  if (sp[0] != 0 || sp[B] != n) return DHSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b) {
+    if (sp[b + 1] < sp[b]) return DHSA_ERR_INVALID_ARG;
+    if (bd[sp[b]] != cu[b] || bd[sp[b + 1]] != cu[b + 1]) return DHSA_ERR_INVALID_ARG;  // no chunk crosses a sequence
+  }
+  return DHSA_OK;
+}
+
+int max_chunks_per_seq(const dhsa_problem* p) {
+  int m = 0;
+  for (int b = 0; b < p->num_seqs; ++b) {
+    const int c = p->h_seq_chunk_ptr[b + 1] - p->h_seq_chunk_ptr[b];
+    if (c > m) m = c;
+  }
+  return m;
+}
+
+int max_chunk_len(const dhsa_problem* p) {
+  int m = 0;
+  for (int c = 0; c < p->num_chunks; ++c) {
+    const int L = p->h_chunk_bounds[c + 1] - p->h_chunk_bounds[c];
+    if (L > m) m = L;
+  }
+  return m;
+}
+
+int64_t nnz_per_head(const dhsa_problem* p, const dhsa_budget& b) {
+  int64_t total = 0;
+  for (int s = 0; s < p->num_seqs; ++s) {
+    const int cnt = p->h_seq_chunk_ptr[s + 1] - p->h_seq_chunk_ptr[s];
+    for (int l = 0; l < cnt; ++l) total += budget_of(l, b) + 1;
+  }
+  return total;
+}
+
+struct PlanLayout {
+  size_t qc, kc, scores, total;
+};
+
+PlanLayout plan_layout(const dhsa_problem* p) {
+  PlanLayout L;
+  const size_t n = static_cast<size_t>(p->num_chunks), d = static_cast<size_t>(p->head_dim);
+  L.qc = kStatusBytes;
+  L.kc = L.qc + align_up(static_cast<size_t>(p->num_q_heads) * n * d * 4);
+  L.scores = L.kc + align_up(static_cast<size_t>(p->num_kv_heads) * n * d * 4);
+  L.total = L.scores + align_up(static_cast<size_t>(p->num_q_heads) * n * n * 4);
+  return L;
+}
+
+dhsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DHSA_OK : DHSA_ERR_CUDA; }
+
+BudgetArgs to_args(const dhsa_budget& b) { return BudgetArgs{b.kind, b.k, b.num, b.den}; }
+
+// Selection core shared by dhsa_topk_select and dhsa_plan (after validation).
+dhsa_status run_select(const float* scores, const dhsa_problem* p, const dhsa_budget& budget, int32_t* row_ptr,
+                       int32_t* col, uint32_t* status, cudaStream_t stream) {
+  const int cap = max_chunks_per_seq(p) > 1 ? max_chunks_per_seq(p) - 1 : 1;
+  if (cap > kMaxSelectCandidates) return DHSA_ERR_UNSUPPORTED;
+  const int64_t per_head = nnz_per_head(p, budget);
+  return cuda_status(launch_topk_select(scores, p->num_chunks, p->num_q_heads, p->seq_chunk_ptr, p->num_seqs,
+                                        to_args(budget), row_ptr, col, static_cast<int>(per_head), cap, status,
+                                        stream));
+}
+
+__global__ void timeout_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  __shared__ int abort_flag;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on this barrier: the wait must give up by itself
+  mbar_wait(bar, 0, reinterpret_cast<volatile int*>(&abort_flag), status, limit_ns);
+}
+
+}  // namespace
+
+cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream) {
+  timeout_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace dhsa
+
+using namespace dhsa;
+
+extern "C" {
+
+const char* dhsa_status_string(dhsa_status s) {
+  switch (s) {
+    case DHSA_OK: return "DHSA_OK";
+    case DHSA_ERR_INVALID_ARG: return "DHSA_ERR_INVALID_ARG";
+    case DHSA_ERR_UNSUPPORTED: return "DHSA_ERR_UNSUPPORTED";
+    case DHSA_ERR_WORKSPACE: return "DHSA_ERR_WORKSPACE";
+    case DHSA_ERR_CUDA: return "DHSA_ERR_CUDA";
+    case DHSA_ERR_TIMEOUT: return "DHSA_ERR_TIMEOUT";
+    case DHSA_ERR_DEVICE_CHECK: return "DHSA_ERR_DEVICE_CHECK";
+  }
+  return "DHSA_ERR_UNKNOWN";
+}
+
+dhsa_status dhsa_validate(const dhsa_problem* p, const dhsa_budget* budget) {
+  dhsa_status s = check_problem(p);
+  if (s != DHSA_OK) return s;
+  if (budget != nullptr) return check_budget(*budget);
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_plan_nnz(const dhsa_problem* p, dhsa_budget budget, int64_t* nnz) {
+  dhsa_status s = dhsa_validate(p, &budget);
+  if (s != DHSA_OK) return s;
+  if (nnz == nullptr) return DHSA_ERR_INVALID_ARG;
+  *nnz = nnz_per_head(p, budget) * p->num_q_heads;
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_chunk_reduce(const void* x, int32_t dtype, int32_t total_tokens, int32_t num_heads,
+                              int32_t head_dim, const int32_t* chunk_bounds, int32_t num_chunks, float* out,
+                              void* stream) {
+  if (dtype != DHSA_BF16 && dtype != DHSA_F32) return DHSA_ERR_INVALID_ARG;
+  if (total_tokens < 0 || num_heads < 1 || num_chunks < 0) return DHSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return DHSA_ERR_UNSUPPORTED;
+  if (num_chunks > 65535) return DHSA_ERR_UNSUPPORTED;
+  if (num_chunks == 0) return DHSA_OK;
+  if (x == nullptr || out == nullptr || chunk_bounds == nullptr || !aligned16(x)) return DHSA_ERR_INVALID_ARG;
+  return cuda_status(launch_chunk_reduce(dtype, x, num_heads, out, nullptr, 0, nullptr, head_dim, chunk_bounds,
+                                         num_chunks, static_cast<cudaStream_t>(stream)));
+}
+
+dhsa_status dhsa_chunk_similarity(const float* qc, const float* kc, const dhsa_problem* p, float* scores,
+                                  void* stream) {
+  dhsa_status s = check_problem(p);
+  if (s != DHSA_OK) return s;
+  if (p->num_chunks == 0) return DHSA_OK;
+  if (qc == nullptr || kc == nullptr || scores == nullptr) return DHSA_ERR_INVALID_ARG;
+  return cuda_status(launch_chunk_similarity(qc, kc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
+                                             p->seq_chunk_ptr, p->num_seqs, scores,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+dhsa_status dhsa_topk_select(const float* scores, const dhsa_problem* p, dhsa_budget budget, int32_t* row_ptr,
+                             int32_t* col, int64_t nnz, void* workspace, size_t workspace_bytes, void* stream) {
+  dhsa_status s = dhsa_validate(p, &budget);
+  if (s != DHSA_OK) return s;
+  const int64_t want = nnz_per_head(p, budget) * p->num_q_heads;
+  if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
+  if (p->num_chunks == 0) return DHSA_OK;
+  if (scores == nullptr || row_ptr == nullptr || col == nullptr) return DHSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  return run_select(scores, p, budget, row_ptr, col, status, st);
+}
+
+dhsa_status dhsa_plan_workspace_size(const dhsa_problem* p, dhsa_budget budget, size_t* bytes) {
+  dhsa_status s = dhsa_validate(p, &budget);
+  if (s != DHSA_OK) return s;
+  if (bytes == nullptr) return DHSA_ERR_INVALID_ARG;
+  *bytes = plan_layout(p).total;
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem* p, dhsa_budget budget, int32_t* row_ptr,
+                      int32_t* col, int64_t nnz, void* workspace, size_t workspace_bytes, void* stream) {
+  dhsa_status s = dhsa_validate(p, &budget);
+  if (s != DHSA_OK) return s;
+  const int64_t want = nnz_per_head(p, budget) * p->num_q_heads;
+  if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
+  const PlanLayout L = plan_layout(p);
+  if (workspace == nullptr || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return DHSA_ERR_WORKSPACE;
+  if (p->num_chunks == 0) return DHSA_OK;
+  if (q == nullptr || k == nullptr || row_ptr == nullptr || col == nullptr || !aligned16(q) || !aligned16(k))
+    return DHSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* qc = reinterpret_cast<float*>(ws + L.qc);
+  float* kc = reinterpret_cast<float*>(ws + L.kc);
+  float* scores = reinterpret_cast<float*>(ws + L.scores);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  cudaError_t e = launch_chunk_reduce(p->dtype, q, p->num_q_heads, qc, k, p->num_kv_heads, kc, p->head_dim,
+                                      p->chunk_bounds, p->num_chunks, st);
+  if (e != cudaSuccess) return DHSA_ERR_CUDA;
+  e = launch_chunk_similarity(qc, kc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
+                              p->seq_chunk_ptr, p->num_seqs, scores, st);
+  if (e != cudaSuccess) return DHSA_ERR_CUDA;
+  return run_select(scores, p, budget, row_ptr, col, status, st);
+}
+
+dhsa_status dhsa_attention_workspace_size(const dhsa_problem* p, size_t* bytes) {
+  dhsa_status s = check_problem(p);
+  if (s != DHSA_OK) return s;
+  if (bytes == nullptr) return DHSA_ERR_INVALID_ARG;
+  *bytes = kStatusBytes;
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_attention(const void* q, const void* k, const void* v, const dhsa_problem* p,
+                           const int32_t* row_ptr, const int32_t* col, int64_t nnz, float scale, void* out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  dhsa_status s = check_problem(p);
+  if (s != DHSA_OK) return s;
+  if (nnz < static_cast<int64_t>(p->num_q_heads) * p->num_chunks) return DHSA_ERR_INVALID_ARG;  // >= diagonal per row
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
+  if (p->total_tokens == 0 || p->num_chunks == 0) return DHSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || row_ptr == nullptr || col == nullptr)
+    return DHSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DHSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(p->head_dim));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  if (p->dtype == DHSA_F32) {
+    return cuda_status(launch_attention_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                            static_cast<const float*>(v), p->chunk_bounds, p->num_chunks, row_ptr,
+                                            col, p->total_tokens, p->num_q_heads, p->num_kv_heads, p->head_dim,
+                                            scale, static_cast<float*>(out), st));
+  }
+  AttnBf16Args a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.bounds = p->chunk_bounds;
+  a.row_ptr = row_ptr;
+  a.col = col;
+  a.num_chunks = p->num_chunks;
+  a.total_tokens = p->total_tokens;
+  a.num_q_heads = p->num_q_heads;
+  a.num_kv_heads = p->num_kv_heads;
+  a.head_dim = p->head_dim;
+  a.max_chunk_len = max_chunk_len(p);
+  a.scale = scale;
+  a.status = status;
+  return cuda_status(launch_attention_bf16(a, st));
+}
+
+dhsa_status dhsa_workspace_status(const void* workspace, void* stream) {
+  if (workspace == nullptr) return DHSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DHSA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return DHSA_ERR_CUDA;
+  if (word & kDevTimeout) return DHSA_ERR_TIMEOUT;
+  if (word & kDevCheck) return DHSA_ERR_DEVICE_CHECK;
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* stream) {
+  if (workspace == nullptr) return DHSA_ERR_WORKSPACE;
+  if (limit_us < 1 || limit_us > 2000000) return DHSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  return cuda_status(launch_timeout_selftest(status, static_cast<unsigned long long>(limit_us) * 1000ull, st));
+}
+
+}  // extern "C"

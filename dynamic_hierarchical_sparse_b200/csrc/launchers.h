@@ -1,0 +1,67 @@
+// Internal launchers of the DHSA kernels (C++ linkage, not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dhsa {
+
+struct BudgetArgs {
+  int kind;  // 0 = top-k, 1 = fraction
+  int k;
+  int num;
+  int den;
+};
+
+// Step 1. Reduces xa ([T, heads_a, d]) into out_a and, when xb is non-null,
+// xb ([T, heads_b, d]) into out_b, in one launch.  dtype 0 = bf16, 1 = fp32.
+cudaError_t launch_chunk_reduce(int dtype, const void* xa, int heads_a, float* out_a, const void* xb,
+                                int heads_b, float* out_b, int head_dim, const int* bounds,
+                                int num_chunks, cudaStream_t stream);
+
+// Step 2.
+cudaError_t launch_chunk_similarity(const float* qc, const float* kc, int num_q_heads, int num_kv_heads,
+                                    int num_chunks, int head_dim, const int* seq_chunk_ptr,
+                                    int num_seqs, float* scores, cudaStream_t stream);
+
+// Step 3.  key_capacity >= the largest number of admissible candidates of any
+// row (chunks per sequence - 1).
+size_t topk_select_smem_bytes(int key_capacity);
+cudaError_t launch_topk_select(const float* scores, int num_chunks, int num_q_heads,
+                               const int* seq_chunk_ptr, int num_seqs, BudgetArgs budget,
+                               int* row_ptr, int* col, int nnz_per_head, int key_capacity,
+                               uint32_t* status, cudaStream_t stream);
+
+// Step 4, fp32.
+cudaError_t launch_attention_f32(const float* q, const float* k, const float* v, const int* bounds,
+                                 int num_chunks, const int* row_ptr, const int* col, int total_tokens,
+                                 int num_q_heads, int num_kv_heads, int head_dim, float scale, float* out,
+                                 cudaStream_t stream);
+
+// Step 4, bf16 on tcgen05.  h_bounds is the host mirror of bounds (used to
+// size the grid).
+struct AttnBf16Args {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  const int* bounds;
+  const int* row_ptr;
+  const int* col;
+  int num_chunks;
+  int total_tokens;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int max_chunk_len;
+  float scale;
+  uint32_t* status;
+};
+cudaError_t launch_attention_bf16(const AttnBf16Args& a, cudaStream_t stream);
+
+// Diagnostic: a kernel whose only wait can never be satisfied, bounded by limit_ns.
+cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);
+
+}  // namespace dhsa

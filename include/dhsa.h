@@ -1,0 +1,190 @@
+/*
+ * dhsa.h - C ABI of libdhsa.so, the B200 (sm_100a) prefill hot path of
+ * Dynamic Hierarchical Sparse Attention (DHSA).
+ *
+ * The method is described on two pages: "Long-Context Modeling with Dynamic
+ * Hierarchical Sparse Attention for On-Device LLMs" (Abstract, AI Summary) and
+ * "Long-Context Modeling with Dynamic Hierarchical Sparse Attention for
+ * Memory-Constrained LLM Inference" (abstract).  The path has four steps:
+ *
+ *   1. chunk aggregation  dhsa_chunk_reduce      (On-Device page, Abstract:
+ *      length-normalised aggregation, mean scaled by sqrt(chunk length))
+ *   2. chunk similarity   dhsa_chunk_similarity  (On-Device page, Abstract:
+ *      chunk-level similarity scores; dot product of representations)
+ *   3. upsample + select  dhsa_topk_select       (On-Device page, Abstract:
+ *      chunk scores upsampled to token level decide which token interactions
+ *      are kept; Memory-Constrained page: importance estimated per chunk and
+ *      propagated to token interactions, keeping causal dependencies)
+ *   4. sparse attention   dhsa_attention         (causal softmax attention over
+ *      the kept token pairs only)
+ *
+ * dhsa_plan runs steps 1-3 back to back.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Token tensors are packed "THD": q [T, Hq, d], k and v [T, Hkv, d],
+ *   contiguous, row-major, in the problem's dtype (bf16 or fp32), 16-byte
+ *   aligned.  Query head h reads KV head h / (Hq / Hkv).
+ * - Chunks are given by global token offsets chunk_bounds[0..n], strictly
+ *   increasing, chunk_bounds[0] = 0, chunk_bounds[n] = T.  Chunks never cross a
+ *   sequence: chunk_bounds[seq_chunk_ptr[b]] == cu_seqlens[b] for every b.
+ * - Every pointer marked "device" is device memory owned by the caller; every
+ *   pointer marked "host" is host memory owned by the caller, read during the
+ *   call only.  The library allocates nothing: the caller passes workspace.
+ * - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *   means the legacy default stream).  Argument errors are detected on the host
+ *   and returned before anything is launched.  Launch failures return
+ *   DHSA_ERR_CUDA.  Errors found by the kernels themselves (a bounded wait that
+ *   ran out, an index check) are written to a status word at the start of the
+ *   workspace and read with dhsa_workspace_status.
+ * - No C++ exception crosses this interface.  All entry points are reentrant.
+ */
+#ifndef DHSA_H_
+#define DHSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DHSA_API __attribute__((visibility("default")))
+#else
+#define DHSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DHSA_OK = 0,
+  DHSA_ERR_INVALID_ARG = 1,  /* bad shape, pointer, bounds or budget */
+  DHSA_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head_dim 96) */
+  DHSA_ERR_WORKSPACE = 3,    /* workspace missing or too small */
+  DHSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  DHSA_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
+  DHSA_ERR_DEVICE_CHECK = 6  /* a device-side index/consistency check failed */
+} dhsa_status;
+
+typedef enum { DHSA_BF16 = 0, DHSA_F32 = 1 } dhsa_dtype;
+
+typedef enum { DHSA_BUDGET_TOPK = 0, DHSA_BUDGET_FRACTION = 1 } dhsa_budget_kind;
+
+/* Key-chunk budget of one query chunk with i_local earlier chunks in its
+ * sequence (the diagonal chunk is always kept on top of it):
+ *   TOPK:     keep min(k, i_local)
+ *   FRACTION: keep min(i_local, ceil(i_local * num / den)), integer arithmetic
+ * Requires k >= 0, num >= 0, den >= 1. */
+typedef struct {
+  int32_t kind;
+  int32_t k;
+  int32_t num;
+  int32_t den;
+} dhsa_budget;
+
+/* Shapes and chunk structure of one packed batch. */
+typedef struct {
+  int32_t dtype;         /* dhsa_dtype of q, k, v and out */
+  int32_t num_seqs;      /* B >= 0 */
+  int32_t total_tokens;  /* T >= 0 */
+  int32_t num_q_heads;   /* Hq >= 1 */
+  int32_t num_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t head_dim;      /* d in {64, 128, 256} */
+  int32_t num_chunks;    /* n >= 0 */
+  const int32_t* cu_seqlens;       /* device [B+1] */
+  const int32_t* chunk_bounds;     /* device [n+1] */
+  const int32_t* seq_chunk_ptr;    /* device [B+1] */
+  const int32_t* h_cu_seqlens;     /* host mirror [B+1] */
+  const int32_t* h_chunk_bounds;   /* host mirror [n+1] */
+  const int32_t* h_seq_chunk_ptr;  /* host mirror [B+1] */
+} dhsa_problem;
+
+/* Human-readable name of a status code (static storage). */
+DHSA_API const char* dhsa_status_string(dhsa_status s);
+
+/* Host-only checks of the problem (and budget when `budget` is non-NULL).
+ * Returns DHSA_OK or the first error found. */
+DHSA_API dhsa_status dhsa_validate(const dhsa_problem* p, const dhsa_budget* budget);
+
+/* Number of plan entries: sum over query heads and chunks of (budget + 1).
+ * Host-only, from the host mirrors.  The plan's row count is Hq * n. */
+DHSA_API dhsa_status dhsa_plan_nnz(const dhsa_problem* p, dhsa_budget budget, int64_t* nnz);
+
+/* ---- step 1: length-normalised chunk aggregation --------------------------
+ * out[h, c, :] = (sum over tokens t of chunk c of x[t, h, :]) / sqrt(L_c),
+ * i.e. the chunk mean scaled by sqrt(L_c) (On-Device page, Abstract), with
+ * fp32 accumulation.
+ *   x     device [T, H, d] in `dtype`
+ *   out   device fp32 [H, n, d]
+ * Deterministic (fixed summation order). */
+DHSA_API dhsa_status dhsa_chunk_reduce(const void* x, int32_t dtype, int32_t total_tokens,
+                              int32_t num_heads, int32_t head_dim,
+                              const int32_t* chunk_bounds, int32_t num_chunks,
+                              float* out, void* stream);
+
+/* ---- step 2: chunk similarity -------------------------------------------
+ * scores[h, i, j] = qc[h, i, :] . kc[h / (Hq/Hkv), j, :] for every j <= i in
+ * the same sequence (On-Device page, Abstract: chunk-level similarity scores).
+ * Entries outside that causal, same-sequence triangle are not written.
+ *   qc      device fp32 [Hq, n, d]
+ *   kc      device fp32 [Hkv, n, d]
+ *   scores  device fp32 [Hq, n, n] */
+DHSA_API dhsa_status dhsa_chunk_similarity(const float* qc, const float* kc,
+                                  const dhsa_problem* p, float* scores,
+                                  void* stream);
+
+/* ---- step 3: upsample + select ------------------------------------------
+ * For each row r = h * n + i: keep the budget's number of admissible key
+ * chunks j < i of i's sequence with the largest scores[h, i, j] (ties to the
+ * lower j), plus the diagonal i.  Because every token pair of chunks (i, j)
+ * inherits score(i, j), this is the token-level keep set of the pages'
+ * upsampling step, stored per chunk.
+ *   row_ptr  device int32 [Hq*n + 1]  (CSR offsets, written)
+ *   col      device int32 [nnz]       (ascending chunk ids; the diagonal is
+ *                                      the last entry of its row)
+ *   nnz      must equal dhsa_plan_nnz() for the same problem and budget. */
+DHSA_API dhsa_status dhsa_topk_select(const float* scores, const dhsa_problem* p,
+                             dhsa_budget budget, int32_t* row_ptr, int32_t* col,
+                             int64_t nnz, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* ---- steps 1-3 ------------------------------------------------------------
+ * Workspace: dhsa_plan_workspace_size bytes, 256-byte aligned, device.  It
+ * holds the status word, qc, kc and the score matrix. */
+DHSA_API dhsa_status dhsa_plan_workspace_size(const dhsa_problem* p, dhsa_budget budget,
+                                     size_t* bytes);
+DHSA_API dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem* p,
+                      dhsa_budget budget, int32_t* row_ptr, int32_t* col,
+                      int64_t nnz, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* ---- step 4: sparse causal attention --------------------------------------
+ * out[t, h, :] = sum over kept s of softmax_s(q[t,h].k[s,g] * scale) v[s,g],
+ * kept s = {s <= t : chunk(s) in row (h, chunk(t)) of the plan}, g = h/(Hq/Hkv).
+ * scale <= 0 selects 1/sqrt(d).  bf16 runs on tcgen05 tensor cores with fp32
+ * accumulation and an fp32 online softmax; fp32 runs an fp32 kernel.
+ *   q, k, v  device, THD, `dtype`; out device [T, Hq, d] in `dtype`
+ *   row_ptr, col: a plan as written by dhsa_plan / dhsa_topk_select
+ * Workspace: dhsa_attention_workspace_size bytes (status word + schedule). */
+DHSA_API dhsa_status dhsa_attention_workspace_size(const dhsa_problem* p, size_t* bytes);
+DHSA_API dhsa_status dhsa_attention(const void* q, const void* k, const void* v,
+                           const dhsa_problem* p, const int32_t* row_ptr,
+                           const int32_t* col, int64_t nnz, float scale, void* out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Waits for `stream`, then reads the status word that the kernels of the last
+ * call given `workspace` may have set.  Returns DHSA_OK, DHSA_ERR_TIMEOUT or
+ * DHSA_ERR_DEVICE_CHECK (or DHSA_ERR_CUDA if the wait itself failed). */
+DHSA_API dhsa_status dhsa_workspace_status(const void* workspace, void* stream);
+
+/* Diagnostic: launches one tiny kernel whose only wait is on a barrier that
+ * nothing releases, with a limit of `limit_us` microseconds (1..2000000); the
+ * kernel gives up, records DHSA_ERR_TIMEOUT in the status word at the start
+ * of `workspace` (>= 256 bytes) and returns.  Exercises the timeout path of
+ * the bounded waits without hanging the device. */
+DHSA_API dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DHSA_H_ */

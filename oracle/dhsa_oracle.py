@@ -29,7 +29,8 @@ abstract):
    selecting the best tokens by upsampled score keeps whole chunks;
    ``attention_literal`` re-derives the keep set from the materialised
    token-level score matrix to check that equivalence.
-4. ``attention_gather`` / ``attention_literal`` / ``attention_rows``: causal
+4. ``attention_query_chunk`` / ``attention_gather`` / ``attention_literal`` /
+   ``attention_rows``: causal
    softmax attention of each query token over the kept key tokens only.
 
 Readings taken where the pages are silent (each listed in the design notes):
@@ -195,35 +196,47 @@ def _softmax_rows(logits: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
-def attention_gather(q, k, v, chunk_bounds, row_ptr, col, scale: Optional[float] = None,
-                     heads: Optional[Iterable[int]] = None) -> np.ndarray:
-    """Sparse causal attention, chunk-gather form.
+def attention_query_chunk(q, k, v, chunk_bounds, row_ptr, col, h: int, i: int,
+                          scale: Optional[float] = None) -> np.ndarray:
+    """Sparse causal attention of the tokens of query chunk i, head h.
 
-    For query chunk i of head h, the kept key chunks' tokens are concatenated;
-    each query token t attends to the kept tokens s <= t with softmax weights of
-    q_t . k_s * scale and averages v_s.  Returns O [T, Hq, d] float64 (rows of
-    heads not listed in ``heads`` are left zero).
+    The kept key chunks' tokens (plan row h*n+i) are concatenated; each query
+    token t attends to the kept tokens s <= t with softmax weights of
+    q_t . k_s * scale and averages v_s.  Returns [L_i, d] float64.
     """
-    q64, k64, v64 = as_f64(q), as_f64(k), as_f64(v)
-    T, Hq, d = q64.shape
-    Hkv = k64.shape[1]
-    group = Hq // Hkv
+    Hq, d = q.shape[1], q.shape[2]
+    group = Hq // k.shape[1]
+    g = h // group
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bounds = np.asarray(chunk_bounds, dtype=np.int64)
     n = bounds.shape[0] - 1
     rp = np.asarray(row_ptr, dtype=np.int64)
     cl = np.asarray(col, dtype=np.int64)
+    kept = cl[rp[h * n + i]:rp[h * n + i + 1]]
+    key_tok = np.concatenate([np.arange(bounds[j], bounds[j + 1]) for j in kept])
+    qs = np.arange(bounds[i], bounds[i + 1])
+    qq = as_f64(q[int(bounds[i]):int(bounds[i + 1]), h, :])
+    kk = as_f64(k[:, g, :][key_tok])
+    vv = as_f64(v[:, g, :][key_tok])
+    logits = (qq @ kk.T) * scale
+    logits = np.where(key_tok[None, :] <= qs[:, None], logits, -np.inf)
+    return _softmax_rows(logits) @ vv
+
+
+def attention_gather(q, k, v, chunk_bounds, row_ptr, col, scale: Optional[float] = None,
+                     heads: Optional[Iterable[int]] = None) -> np.ndarray:
+    """Sparse causal attention, chunk-gather form, for every query chunk.
+
+    Returns O [T, Hq, d] float64 (rows of heads not in ``heads`` stay zero).
+    """
+    T, Hq, d = q.shape
+    bounds = np.asarray(chunk_bounds, dtype=np.int64)
+    n = bounds.shape[0] - 1
     out = np.zeros((T, Hq, d), dtype=np.float64)
     for h in (range(Hq) if heads is None else heads):
-        g = h // group
         for i in range(n):
-            kept = cl[rp[h * n + i]:rp[h * n + i + 1]]
-            key_tok = np.concatenate([np.arange(bounds[j], bounds[j + 1]) for j in kept])
-            qs = np.arange(bounds[i], bounds[i + 1])
-            logits = (q64[qs, h, :] @ k64[key_tok, g, :].T) * scale
-            logits = np.where(key_tok[None, :] <= qs[:, None], logits, -np.inf)
-            p = _softmax_rows(logits)
-            out[qs, h, :] = p @ v64[key_tok, g, :]
+            out[bounds[i]:bounds[i + 1], h, :] = attention_query_chunk(q, k, v, bounds, row_ptr, col, h, i,
+                                                                       scale)
     return out
 
 

@@ -1,0 +1,175 @@
+"""GPU parity: every step of the CUDA path against the fp64 oracle, through the C ABI.
+
+Sizes are small enough for the oracle to finish in seconds, yet span several
+tiles and ragged tails (chunk lengths 1, 2, 17, 127..129, 255..300).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_hierarchical_sparse_b200 import api, workloads as W
+from oracle import dhsa_oracle as O
+from tests.helpers import (attention_gate, compare_plans, gpu_rows, reduce_bound, to_device)
+
+pytestmark = pytest.mark.gpu
+
+RAGGED_LENS = [[1, 2, 17, 127, 128, 129, 60, 255, 3, 300], [64, 1, 190, 45], [7]]
+
+
+def _case(name):
+    if name == "ragged_d128_top2":
+        return W.explicit_problem(0, RAGGED_LENS, 4, 2, 128, "bf16", W.Budget.topk(2))
+    if name == "ragged_d64_frac":
+        return W.explicit_problem(1, RAGGED_LENS, 2, 1, 64, "bf16", W.Budget.fraction(1, 3))
+    if name == "d256_structured_top3":
+        return W.random_problem(2, [1500], 4, 2, 256, "bf16", 64, 256, W.Budget.topk(3), "structured")
+    if name == "d128_dense":
+        return W.random_problem(3, [900, 400], 4, 1, 128, "bf16", 30, 200, W.Budget.topk(10 ** 6))
+    if name == "d128_diag_only":
+        return W.random_problem(4, [1000], 2, 2, 128, "bf16", 50, 300, W.Budget.topk(0))
+    if name == "d128_long_runs":
+        return W.random_problem(5, [3000], 2, 1, 128, "bf16", 128, 512, W.Budget.fraction(1, 2), "structured")
+    if name == "tiny_f32":
+        return W.generate(W.TINY_1K_F32, 0)
+    if name == "f32_d128_ragged":
+        return W.explicit_problem(6, RAGGED_LENS, 2, 1, 128, "f32", W.Budget.topk(3))
+    raise KeyError(name)
+
+
+CASES = ["ragged_d128_top2", "ragged_d64_frac", "d256_structured_top3", "d128_dense", "d128_diag_only",
+         "d128_long_runs", "tiny_f32", "f32_d128_ragged"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    api.lib()
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_chunk_reduce(name):
+    inp = _case(name)
+    q, k, v, prob = to_device(inp)
+    for x in (inp.q, inp.k):
+        got = api.chunk_reduce(x.cuda(), prob).double().cpu().numpy()
+        want = O.chunk_representations(x, inp.chunk_bounds)
+        bound = reduce_bound(x, inp.chunk_bounds)
+        assert np.all(np.abs(got - want) <= bound), float(np.max(np.abs(got - want) - bound))
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_chunk_similarity(name):
+    """Same fp32 representations in; fp32 dot products out, within the fp32 bound."""
+    inp = _case(name)
+    _, _, _, prob = to_device(inp)
+    qc = O.chunk_representations(inp.q, inp.chunk_bounds).astype(np.float32)
+    kc = O.chunk_representations(inp.k, inp.chunk_bounds).astype(np.float32)
+    got = api.chunk_similarity(torch.from_numpy(qc).cuda(), torch.from_numpy(kc).cuda(), prob).double().cpu().numpy()
+    want = O.chunk_scores(qc.astype(np.float64), kc.astype(np.float64), inp.seq_chunk_ptr)
+    d = qc.shape[2]
+    group = qc.shape[0] // kc.shape[0]
+    absdot = np.einsum("hid,hjd->hij", np.abs(qc.astype(np.float64)),
+                       np.abs(np.repeat(kc.astype(np.float64), group, axis=0)))
+    mask = ~np.isnan(want)
+    err = np.abs(got - np.nan_to_num(want))[mask]
+    assert np.all(err <= (d + 2) * 2.0 ** -24 * absdot[mask] + 1e-30)
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_topk_select_bit_exact_on_same_scores(name):
+    """Selection from identical fp32 scores is integer work: bit-exact."""
+    inp = _case(name)
+    _, _, _, prob = to_device(inp)
+    qc = O.chunk_representations(inp.q, inp.chunk_bounds).astype(np.float32)
+    kc = O.chunk_representations(inp.k, inp.chunk_bounds).astype(np.float32)
+    S32 = api.chunk_similarity(torch.from_numpy(qc).cuda(), torch.from_numpy(kc).cuda(), prob)
+    # plant exact ties: copy a score onto its neighbour in a few rows
+    S32 = S32.clone()
+    n = inp.num_chunks
+    for i in range(2, n, 3):
+        S32[:, i, i - 1] = S32[:, i, i - 2]
+    plan = api.topk_select(S32, prob, inp.budget, check=True)
+    S = S32.double().cpu().numpy()
+    b = inp.budget
+    ptr = inp.seq_chunk_ptr
+    rows = gpu_rows(plan, inp.spec.num_q_heads * n)
+    for h in range(inp.spec.num_q_heads):
+        for bb in range(len(ptr) - 1):
+            for i in range(int(ptr[bb]), int(ptr[bb + 1])):
+                cand = list(range(int(ptr[bb]), i))
+                keep = O.row_budget(i - int(ptr[bb]), b.kind, b.k, b.num, b.den)
+                want = sorted(O.select_row([S[h, i, j] for j in cand], cand, keep)) + [i]
+                assert rows[h * n + i] == want, (h, i)
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_plan_and_attention(name):
+    inp = _case(name)
+    q, k, v, prob = to_device(inp)
+    b = inp.budget
+    plan = api.plan(q, k, prob, b, check=True)
+    ref = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, b.kind, b.k, b.num, b.den)
+    rows = gpu_rows(plan, inp.spec.num_q_heads * inp.num_chunks)
+    tolerated = compare_plans(rows, ref, inp, b)
+    assert len(tolerated) <= max(2, len(rows) // 100)
+    out = api.attention(q, k, v, prob, plan, check=True)
+    torch.cuda.synchronize()
+    want = O.attention_gather(inp.q, inp.k, inp.v, inp.chunk_bounds, plan.row_ptr.cpu().numpy(),
+                              plan.col.cpu().numpy())
+    stats = attention_gate(out, want, inp.q.dtype)
+    print(name, "max_err=%.3g max|O|=%.3g median|O|=%.3g rel_fro=%.3g" % stats)
+
+
+def test_dense_budget_matches_sdpa():
+    inp = _case("d128_dense")
+    q, k, v, prob = to_device(inp)
+    plan = api.plan(q, k, prob, inp.budget)
+    out = api.attention(q, k, v, prob, plan, check=True).float()
+    ref = torch.empty_like(out)
+    cu = inp.cu_seqlens
+    for bb in range(len(cu) - 1):
+        s, e = int(cu[bb]), int(cu[bb + 1])
+        qq = q[s:e].float().transpose(0, 1)[None]
+        kk = k[s:e].float().transpose(0, 1).repeat_interleave(4, 0)[None]
+        vv = v[s:e].float().transpose(0, 1).repeat_interleave(4, 0)[None]
+        ref[s:e] = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True)[0].transpose(0, 1)
+    assert float((out - ref).abs().max()) <= 2e-2
+
+
+def test_custom_scale_and_repeat_calls_are_deterministic():
+    inp = _case("ragged_d128_top2")
+    q, k, v, prob = to_device(inp)
+    plan = api.plan(q, k, prob, inp.budget)
+    plan2 = api.plan(q, k, prob, inp.budget)
+    assert torch.equal(plan.col, plan2.col) and torch.equal(plan.row_ptr, plan2.row_ptr)
+    o1 = api.attention(q, k, v, prob, plan, scale=0.05)
+    o2 = api.attention(q, k, v, prob, plan, scale=0.05)
+    assert torch.equal(o1, o2)
+    want = O.attention_gather(inp.q, inp.k, inp.v, inp.chunk_bounds, plan.row_ptr.cpu().numpy(),
+                              plan.col.cpu().numpy(), scale=0.05)
+    attention_gate(o1, want, torch.bfloat16)
+
+
+def test_empty_sequence_in_batch():
+    inp = W.random_problem(7, [500, 0, 300], 2, 1, 64, "bf16", 40, 120, W.Budget.topk(2))
+    q, k, v, prob = to_device(inp)
+    plan = api.plan(q, k, prob, inp.budget, check=True)
+    ref = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, O.TOPK, 2)
+    compare_plans(gpu_rows(plan, 2 * inp.num_chunks), ref, inp, inp.budget)
+    out = api.attention(q, k, v, prob, plan, check=True)
+    want = O.attention_gather(inp.q, inp.k, inp.v, inp.chunk_bounds, plan.row_ptr.cpu().numpy(),
+                              plan.col.cpu().numpy())
+    attention_gate(out, want, torch.bfloat16)
+
+
+def test_timeout_path_reports_and_context_survives():
+    assert api.selftest_timeout(20000) == 5  # DHSA_ERR_TIMEOUT
+    inp = _case("d128_diag_only")
+    q, k, v, prob = to_device(inp)
+    plan = api.plan(q, k, prob, inp.budget, check=True)
+    api.attention(q, k, v, prob, plan, check=True)
+    torch.cuda.synchronize()

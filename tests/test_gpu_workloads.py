@@ -1,0 +1,77 @@
+"""GPU parity at the five named workloads' full sizes, in the launch
+configuration the benchmark times: the whole plan against the oracle's plan
+(bit-exact under the near-tie rule) and attention on sampled (token, head)
+rows computed one by one by the oracle.  The ragged workload also checks that
+every planted needle chunk is selected."""
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_hierarchical_sparse_b200 import api, workloads as W
+from oracle import dhsa_oracle as O
+from tests.helpers import ATOL_BF16, ATOL_F32, compare_plans, gpu_rows, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    api.lib()
+
+
+def _sample_rows(inp, count, seed):
+    rng = np.random.default_rng(seed)
+    T = int(inp.cu_seqlens[-1])
+    Hq = inp.spec.num_q_heads
+    b = inp.chunk_bounds
+    rows = set()
+    # chunk edges and sequence ends, spread over heads
+    for c in rng.choice(inp.num_chunks, size=min(inp.num_chunks, count // 4), replace=False):
+        rows.add((int(b[c]), int(rng.integers(Hq))))
+        rows.add((int(b[c + 1]) - 1, int(rng.integers(Hq))))
+    for e in inp.cu_seqlens[1:]:
+        rows.add((int(e) - 1, Hq - 1))
+    while len(rows) < count:
+        rows.add((int(rng.integers(T)), int(rng.integers(Hq))))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("spec", W.WORKLOADS, ids=[w.name for w in W.WORKLOADS])
+def test_workload_full_size(spec):
+    inp = W.generate(spec, 0)
+    q, k, v, prob = to_device(inp)
+    b = inp.budget
+    planner = api.Planner(prob, b)
+    attn = api.Attention(prob)
+    plan = planner(q, k)
+    out = torch.empty_like(q)
+    attn(q, k, v, plan, out)
+    assert planner.status() == 0 and attn.status() == 0
+    torch.cuda.synchronize()
+
+    ref = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, b.kind, b.k, b.num, b.den)
+    rows = gpu_rows(plan, spec.num_q_heads * inp.num_chunks)
+    tolerated = compare_plans(rows, ref, inp, b)
+    print(spec.name, "plan rows:", len(rows), "near-tie rows:", len(tolerated))
+    assert len(tolerated) <= max(2, len(rows) // 200)
+
+    if inp.needle_chunks is not None:
+        n = inp.num_chunks
+        group = spec.num_q_heads // spec.num_kv_heads
+        for bb, jstar in enumerate(inp.needle_chunks):
+            last = int(inp.seq_chunk_ptr[bb + 1]) - 1
+            for g in range(spec.num_kv_heads):
+                assert jstar in rows[g * group * n + last], (bb, g)
+
+    sample = _sample_rows(inp, 96 if spec.dtype == "bf16" else 256, 1)
+    want = O.attention_rows(inp.q, inp.k, inp.v, inp.chunk_bounds, plan.row_ptr.cpu().numpy(),
+                            plan.col.cpu().numpy(), sample)
+    got = torch.stack([out[t, h] for (t, h) in sample]).double().cpu().numpy()
+    err = np.abs(got - want)
+    tol = ATOL_BF16 if spec.dtype == "bf16" else ATOL_F32
+    print(spec.name, "sampled rows:", len(sample), "max_err=%.3g max|O|=%.3g median|O|=%.3g"
+          % (err.max(), np.abs(want).max(), np.median(np.abs(want))))
+    assert err.max() <= tol

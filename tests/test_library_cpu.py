@@ -1,0 +1,186 @@
+"""CPU-only checks of the C-ABI library: it builds, loads, exports every symbol
+the header declares, and validates arguments on the host (no kernel runs)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_hierarchical_sparse_b200 import api, build, workloads as W
+from oracle import dhsa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CPU = torch.device("cpu")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "dhsa.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"DHSA_API\s+[\w\s\*]+?\b(dhsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared_symbols() == sorted(api.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(api.library_path())
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+    # nothing else with C linkage leaks out under the dhsa_ prefix
+    out = os.popen("nm -D --defined-only %s" % api.library_path()).read()
+    exported = sorted(set(re.findall(r"\bT (dhsa_\w+)", out)))
+    assert exported == _declared_symbols()
+
+
+def test_status_strings():
+    L = api.lib()
+    for code, name in api.STATUS_NAMES.items():
+        assert L.dhsa_status_string(code).decode() == name
+
+
+def _problem(inp, **over):
+    s = inp.spec
+    kw = dict(num_q_heads=s.num_q_heads, num_kv_heads=s.num_kv_heads, head_dim=s.head_dim,
+              dtype=inp.q.dtype)
+    kw.update(over)
+    return api.Problem(inp.cu_seqlens, inp.chunk_bounds, inp.seq_chunk_ptr, device=CPU, **kw)
+
+
+@pytest.mark.parametrize("budget", [W.Budget.topk(0), W.Budget.topk(3), W.Budget.topk(10 ** 6),
+                                    W.Budget.fraction(1, 10), W.Budget.fraction(1, 20),
+                                    W.Budget.fraction(3, 2)])
+def test_plan_nnz_matches_oracle_row_budget(budget):
+    inp = W.random_problem(0, [700, 33, 1500], 4, 2, 64, "bf16", 16, 80, budget)
+    p = _problem(inp)
+    ptr = inp.seq_chunk_ptr
+    per_head = 0
+    for b in range(len(ptr) - 1):
+        for il in range(ptr[b + 1] - ptr[b]):
+            per_head += O.row_budget(il, budget.kind, budget.k, budget.num, budget.den) + 1
+    assert p.nnz(budget) == 4 * per_head
+
+
+def test_workspace_sizes():
+    inp = W.random_problem(0, [2048], 8, 2, 128, "bf16", 64, 256, W.Budget.topk(4))
+    p = _problem(inp)
+    n = inp.num_chunks
+    ws = p.plan_workspace_bytes(W.Budget.topk(4))
+    need = 256 + (8 * n * 128 + 2 * n * 128 + 8 * n * n) * 4
+    assert need <= ws <= need + 4 * 256
+    assert p.attention_workspace_bytes() >= 256
+
+
+def _code(problem, budget=None):
+    return problem.validate(budget)
+
+
+def test_validation_accepts_good_problems():
+    for spec in [W.TINY_1K_F32, W.RAGGED_NEEDLE]:
+        inp = W.generate(spec, 0, seq_lens=[256, 512] if spec.needle else None)
+        assert _code(_problem(inp), spec.budget) == 0
+
+
+@pytest.mark.parametrize("case", ["gqa", "head_dim", "head_dim_neg", "budget_k", "budget_den",
+                                  "bounds_order", "bounds_cover", "cross_seq", "seqptr"])
+def test_validation_rejects(case):
+    inp = W.random_problem(1, [300, 200], 4, 2, 64, "bf16", 20, 60, W.Budget.topk(2))
+    budget = W.Budget.topk(2)
+    bounds = inp.chunk_bounds.copy()
+    sptr = inp.seq_chunk_ptr.copy()
+    cu = inp.cu_seqlens.copy()
+    kw = {}
+    want = 1
+    if case == "gqa":
+        kw = dict(num_q_heads=6, num_kv_heads=4)
+    elif case == "head_dim":
+        kw = dict(head_dim=96)
+        want = 2
+    elif case == "head_dim_neg":
+        kw = dict(head_dim=0)
+    elif case == "budget_k":
+        budget = W.Budget.topk(-1)
+    elif case == "budget_den":
+        budget = W.Budget.fraction(1, 0)
+    elif case == "bounds_order":
+        bounds[2], bounds[3] = bounds[3], bounds[2]
+    elif case == "bounds_cover":
+        bounds[-1] -= 1
+    elif case == "cross_seq":
+        # move the sequence edge inside a chunk
+        cu[1] += 1
+    elif case == "seqptr":
+        sptr[1] = sptr[1] + 1
+    s = inp.spec
+    args = dict(num_q_heads=s.num_q_heads, num_kv_heads=s.num_kv_heads, head_dim=s.head_dim,
+                dtype=inp.q.dtype)
+    args.update(kw)
+    p = api.Problem(cu, bounds, sptr, device=CPU, **args)
+    assert _code(p, budget) == want
+
+
+def test_entry_points_reject_before_launch():
+    """Invalid calls return their error code without touching the (absent) GPU."""
+    inp = W.random_problem(2, [300], 2, 1, 64, "bf16", 20, 60, W.Budget.topk(2))
+    p = _problem(inp)
+    L = api.lib()
+    b = api._budget(W.Budget.topk(2))
+    nnz = p.nnz(W.Budget.topk(2))
+    null = ctypes.c_void_p(0)
+    ws = ctypes.c_void_p(256)
+    # wrong nnz
+    assert L.dhsa_plan(ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(), b, ctypes.c_void_p(16),
+                       ctypes.c_void_p(16), nnz + 1, ws, 1 << 30, null) == 1
+    # too little workspace
+    assert L.dhsa_plan(ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(), b, ctypes.c_void_p(16),
+                       ctypes.c_void_p(16), nnz, ws, 16, null) == 3
+    # misaligned q
+    assert L.dhsa_attention(ctypes.c_void_p(17), ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(),
+                            ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ctypes.c_float(0.0),
+                            ctypes.c_void_p(16), ws, 256, null) == 1
+    # missing workspace
+    assert L.dhsa_attention(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(),
+                            ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ctypes.c_float(0.0),
+                            ctypes.c_void_p(16), null, 0, null) == 3
+    # timeout self-test limits
+    assert L.dhsa_selftest_timeout(ws, 0, null) == 1
+    assert L.dhsa_selftest_timeout(null, 100, null) == 3
+
+
+def test_empty_problem_is_a_no_op():
+    p = api.Problem([0], [0], [0], 4, 2, 128, torch.bfloat16, device=CPU)
+    assert p.validate(W.Budget.topk(3)) == 0
+    assert p.nnz(W.Budget.topk(3)) == 0
+    L = api.lib()
+    null = ctypes.c_void_p(0)
+    ws = ctypes.c_void_p(256)
+    assert L.dhsa_plan(null, null, p.ref(), api._budget(W.Budget.topk(3)), null, null, 0, ws,
+                       p.plan_workspace_bytes(W.Budget.topk(3)), null) == 0
+    assert L.dhsa_attention(null, null, null, p.ref(), null, null, 0, ctypes.c_float(0.0), null, ws, 256,
+                            null) == 0
+
+
+def test_product_path_has_no_cpu_fallback(monkeypatch):
+    """Without the library the binding raises instead of computing anything."""
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "_LIB_PATH", "/nonexistent/libdhsa.so")
+    with pytest.raises(RuntimeError):
+        api.lib()
+
+
+def test_product_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "dynamic_hierarchical_sparse_b200")
+    pat = re.compile(r"^\s*(from\s+oracle|import\s+oracle)|dhsa_oracle", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    assert not pat.search(f.read()), fn
