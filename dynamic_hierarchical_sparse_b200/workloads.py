@@ -20,8 +20,9 @@ Recipe (one generator per quantity, all seeded):
 * the "structured" value mix is ``X = Z + 2 * A @ B`` with ``Z, A, B ~ N(0,1)``,
   ``A`` of shape ``[T, 4]`` drawn per tensor and per head, ``B`` of shape
   ``[4, d]`` shared by the query heads of a KV group and that group's K head
-  (V draws its own ``B``).  The shared rank-4 part gives hub ("sink-like")
-  keys and peaky attention rows, so outputs are O(1);
+  (V draws its own ``B`` and is divided by sqrt(17), its standard deviation,
+  so outputs are O(1)).  The shared rank-4 part gives hub ("sink-like") keys
+  and peaky attention rows;
 * the ragged workload plants one "needle" key chunk per sequence: every K token
   of a seeded chunk ``j*`` is set, per KV head ``g``, to ``4 * m / |m|`` where
   ``m`` is the mean query (head ``g * Hq/Hkv``) over the sequence's last chunk.
@@ -30,6 +31,7 @@ Recipe (one generator per quantity, all seeded):
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import List, Optional, Sequence
 
 import numpy as np
@@ -196,7 +198,9 @@ def generate(spec: WorkloadSpec, seed: int = 0, seq_lens: Optional[Sequence[int]
         bv = torch.randn(Hkv, 4, d, generator=gen, dtype=torch.float32)
         q = _structured(gen, T, Hq, d, bq, [h // group for h in range(Hq)])
         k = _structured(gen, T, Hkv, d, bq, list(range(Hkv)))
-        v = _structured(gen, T, Hkv, d, bv, list(range(Hkv)))
+        # V at unit per-element variance (Z + 2AB has variance 1 + 16) so that
+        # attention outputs stay O(1), the regime the absolute error gate is for
+        v = _structured(gen, T, Hkv, d, bv, list(range(Hkv))) / math.sqrt(17.0)
     else:
         q = torch.randn(T, Hq, d, generator=gen, dtype=torch.float32)
         k = torch.randn(T, Hkv, d, generator=gen, dtype=torch.float32)
