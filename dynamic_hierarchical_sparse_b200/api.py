@@ -31,7 +31,7 @@ EXPORTED = [
     "dhsa_status_string", "dhsa_validate", "dhsa_plan_nnz", "dhsa_chunk_reduce",
     "dhsa_chunk_similarity", "dhsa_topk_select", "dhsa_plan_workspace_size", "dhsa_plan",
     "dhsa_attention_workspace_size", "dhsa_attention", "dhsa_workspace_status",
-    "dhsa_selftest_timeout",
+    "dhsa_selftest_timeout", "dhsa_plan_noalloc",
 ]
 
 
@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
             "dhsa_attention": (ctypes.c_int, [P, P, P, PP, P, P, I64, ctypes.c_float, P, P, SZ, P]),
             "dhsa_workspace_status": (ctypes.c_int, [P, P]),
             "dhsa_selftest_timeout": (ctypes.c_int, [P, I32, P]),
+            "dhsa_plan_noalloc": (ctypes.c_int, [P, P, PP, _Budget, P, P, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)

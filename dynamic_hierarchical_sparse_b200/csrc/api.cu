@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/dhsa.h"
 #include "common.cuh"
 #include "launchers.h"
@@ -139,6 +141,34 @@ cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_n
   timeout_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
   return cudaGetLastError();
 }
+
+// Fixed scratch of dhsa_plan_noalloc (status word, qc, kc, scores).  Host code
+// must not use this name as a device address: it is a host-side stand-in, so
+// the address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_plan_noalloc_scratch[DHSA_PLAN_NOALLOC_MAX_SCRATCH];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the fixed scratch on the current device (looked up once).
+dhsa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DHSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_plan_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return DHSA_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return DHSA_OK;
+}
+
+}  // namespace
 
 }  // namespace dhsa
 
@@ -306,6 +336,38 @@ dhsa_status dhsa_workspace_status(const void* workspace, void* stream) {
   if (word & kDevTimeout) return DHSA_ERR_TIMEOUT;
   if (word & kDevCheck) return DHSA_ERR_DEVICE_CHECK;
   return DHSA_OK;
+}
+
+dhsa_status dhsa_plan_noalloc(const void* q, const void* k, const dhsa_problem* p, dhsa_budget budget,
+                              int32_t* row_ptr, int32_t* col, int64_t nnz, void* stream) {
+  dhsa_status s = dhsa_validate(p, &budget);
+  if (s != DHSA_OK) return s;
+  const int64_t want = nnz_per_head(p, budget) * p->num_q_heads;
+  if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
+  const PlanLayout L = plan_layout(p);
+  if (L.total > DHSA_PLAN_NOALLOC_MAX_SCRATCH) return DHSA_ERR_WORKSPACE;  // problem too large for the fixed scratch
+  if (p->num_chunks == 0) return DHSA_OK;
+  if (q == nullptr || k == nullptr || row_ptr == nullptr || col == nullptr || !aligned16(q) || !aligned16(k))
+    return DHSA_ERR_INVALID_ARG;
+  void* base = nullptr;
+  s = noalloc_scratch(&base);
+  if (s != DHSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(base);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* qc = reinterpret_cast<float*>(ws + L.qc);
+  float* kc = reinterpret_cast<float*>(ws + L.kc);
+  float* scores = reinterpret_cast<float*>(ws + L.scores);
+  // qc, kc and the score triangle are fully rewritten before they are read;
+  // only the status word has to start at zero
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  cudaError_t e = launch_chunk_reduce(p->dtype, q, p->num_q_heads, qc, k, p->num_kv_heads, kc, p->head_dim,
+                                      p->chunk_bounds, p->num_chunks, st);
+  if (e != cudaSuccess) return DHSA_ERR_CUDA;
+  e = launch_chunk_similarity(qc, kc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
+                              p->seq_chunk_ptr, p->num_seqs, scores, st);
+  if (e != cudaSuccess) return DHSA_ERR_CUDA;
+  return run_select(scores, p, budget, row_ptr, col, status, st);
 }
 
 dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* stream) {

@@ -183,6 +183,31 @@ DHSA_API dhsa_status dhsa_workspace_status(const void* workspace, void* stream);
  * the bounded waits without hanging the device. */
 DHSA_API dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* stream);
 
+/* ---- steps 1-3 without a caller workspace ----------------------------------
+ * No counterpart in the paper: an interface addition for callers that cannot
+ * allocate device memory at the point where they plan, such as code that runs
+ * inside another framework's allocator-free region, a plugin that is handed
+ * only its input and output buffers, or a process whose allocations go through
+ * a pool it does not own.  Same inputs, outputs and results as dhsa_plan; the
+ * scratch (status word, qc, kc, score matrix) lives in one fixed device array
+ * inside the library, DHSA_PLAN_NOALLOC_MAX_SCRATCH bytes per device, which
+ * every GPU that loads the library holds until the process exits.
+ * - Problems whose plan scratch (dhsa_plan_workspace_size) exceeds that size
+ *   are rejected with DHSA_ERR_WORKSPACE before anything is launched.
+ * - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture on the device.
+ * - All calls share the one array and leave their intermediates in it.  Calls
+ *   whose kernels overlap on the GPU (other streams, other threads) race on it
+ *   and give wrong plans: serialise them.
+ * - The array's status word is cleared by each call but cannot be read back;
+ *   device-side consistency checks of this variant are not reported. */
+#define DHSA_PLAN_NOALLOC_MAX_SCRATCH (16u << 20)
+DHSA_API dhsa_status dhsa_plan_noalloc(const void* q, const void* k, const dhsa_problem* p,
+                                       dhsa_budget budget, int32_t* row_ptr, int32_t* col,
+                                       int64_t nnz, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
