@@ -339,6 +339,70 @@ def bench_gpu(args):
         print(json.dumps(result), flush=True)
 
 
+SELECT_MICRO = W.WorkloadSpec(
+    "select_micro_128k_h32_chunks16to64_frac5", [131072], 32, 8, 128, "bf16", 16, 64,
+    W.Budget.fraction(1, 20), "normal")
+
+
+def select_micro_inputs(seed: int = 0):
+    """Chunk structure of the select micro-benchmark (no token tensors needed)."""
+    rng = np.random.default_rng(seed)
+    lens = W.chunk_lengths_until(rng, SELECT_MICRO.seq_lens[0], SELECT_MICRO.chunk_lo, SELECT_MICRO.chunk_hi)
+    return W.make_bounds(SELECT_MICRO.seq_lens, [lens])
+
+
+def triangle_bytes(seq_chunk_ptr, num_q_heads):
+    ptr = np.asarray(seq_chunk_ptr, dtype=np.int64)
+    m = np.diff(ptr)
+    return int(num_q_heads * (m * (m - 1) // 2).sum() * 4)
+
+
+def bench_select_micro(args):
+    """Step 3 alone at a size where its bytes matter: T=131072, 32 heads,
+    chunk lengths U[16,64] (n ~ 3300), keep 5 % + diagonal, fp32 scores
+    drawn N(0,1) on the device.  Reports achieved GB/s on the algorithmic bytes
+    (causal score triangle read + plan written) against measured HBM."""
+    from dynamic_hierarchical_sparse_b200 import api
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cu, bounds, sptr = select_micro_inputs(0)
+    spec = SELECT_MICRO
+    prob = api.Problem(cu, bounds, sptr, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, torch.bfloat16, dev)
+    n = prob.num_chunks
+    gen = torch.Generator(device=dev).manual_seed(0)
+    scores = torch.randn(spec.num_q_heads, n, n, generator=gen, device=dev, dtype=torch.float32)
+    budget = spec.budget
+    plan = api.topk_select(scores, prob, budget, check=True)
+    for _ in range(args.warmup):
+        api.topk_select(scores, prob, budget)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the triangle (0.69 GB) is read once per call and exceeds L2, so calls do not hit in L2
+    e0.record(stream)
+    for _ in range(args.steps):
+        api.topk_select(scores, prob, budget)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / args.steps
+    tri = triangle_bytes(sptr, spec.num_q_heads)
+    out_bytes = (plan.nnz + plan.row_ptr.numel()) * 4
+    gbs = (tri + out_bytes) / t / 1e9
+    peaks = _peaks()
+    print(json.dumps({
+        "metric": "select kernel HBM GB/s (micro-benchmark)", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_call": t * 1e3,
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic N(0,1) scores (seeded, on device)",
+        "config": {"workload": spec.name, "tokens": int(cu[-1]), "q_heads": spec.num_q_heads, "num_chunks": n,
+                   "budget": _budget_str(budget), "nnz": plan.nnz, "triangle_bytes": tri,
+                   "l2": "no flush: triangle %.2f GB > 126 MB L2" % (tri / 1e9)},
+        "roofline": {"kernel": "topk_select_kernel", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "peak_kind": "%s copy bandwidth" % peaks["source"]},
+    }), flush=True)
+
+
 def _budget_str(b):
     if b.kind == W.BUDGET_TOPK:
         return "top-%d + diagonal" % b.k
@@ -380,17 +444,21 @@ def bench_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--micro", default=None, choices=["select"],
+                    help="time one kernel alone instead of the full step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3", file=sys.stderr)
         args.warmup = 3
-    if args.impl == "reference":
+    if args.micro == "select":
+        bench_select_micro(args)
+    elif args.impl == "reference":
         bench_reference(args)
     else:
         bench_gpu(args)

@@ -395,7 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-CUresult encode_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows) {
+}  // namespace
+
+// 3-D (d, heads, tokens) view of a packed THD bf16 tensor with a (64, 1,
+// box_rows) box and 128-byte swizzle: one box lands as box_rows x 128 bytes,
+// the canonical K-major SW128 operand layout of tcgen05.mma.
+CUresult encode_qkv_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows) {
   using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -419,13 +424,15 @@ CUresult encode_map(CUtensorMap* map, const void* base, int heads, int head_dim,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+namespace {
+
 template <int D, int BN>
 cudaError_t launch_dim(const AttnBf16Args& a, cudaStream_t stream) {
   using C = Cfg<D, BN>;
   CUtensorMap mq, mk, mv;
-  if (encode_map(&mq, a.q, a.num_q_heads, D, a.total_tokens, kBM) != CUDA_SUCCESS ||
-      encode_map(&mk, a.k, a.num_kv_heads, D, a.total_tokens, BN) != CUDA_SUCCESS ||
-      encode_map(&mv, a.v, a.num_kv_heads, D, a.total_tokens, BN) != CUDA_SUCCESS)
+  if (encode_qkv_map(&mq, a.q, a.num_q_heads, D, a.total_tokens, kBM) != CUDA_SUCCESS ||
+      encode_qkv_map(&mk, a.k, a.num_kv_heads, D, a.total_tokens, BN) != CUDA_SUCCESS ||
+      encode_qkv_map(&mv, a.v, a.num_kv_heads, D, a.total_tokens, BN) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   auto kern = attention_bf16_kernel<D, BN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -445,9 +452,8 @@ cudaError_t launch_attention_bf16(const AttnBf16Args& a, cudaStream_t stream) {
   if (a.total_tokens <= 0 || a.num_chunks <= 0) return cudaSuccess;
   switch (a.head_dim) {
     case 64:
-      return launch_dim<64, 128>(a, stream);
     case 128:
-      return launch_dim<128, 128>(a, stream);
+      return launch_attention_pair(a, stream);  // two query tiles per CTA (attention_bf16_pair.cu)
     case 256:
       return launch_dim<256, 64>(a, stream);
     default:

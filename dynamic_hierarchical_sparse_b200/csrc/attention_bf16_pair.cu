@@ -1,0 +1,516 @@
+// Step 4 of the DHSA path for bf16 inputs, head_dim 64 and 128: varlen
+// block-sparse causal flash attention on tcgen05 tensor cores, two query tiles
+// per CTA.
+//
+// out[t, h] = sum_s softmax_s(q[t,h] . k[s,g] * scale) v[s,g] over the kept
+// key tokens s <= t: the tokens of the chunks in plan row (h, chunk(t))
+// ("Long-Context Modeling with Dynamic Hierarchical Sparse Attention for
+// On-Device LLMs", Abstract: only the token interactions selected through the
+// upsampled chunk scores are preserved; "... for Memory-Constrained LLM
+// Inference": causally important dependencies are kept).
+//
+// Work item = one CTA = (query chunk i, head h, pair of 128-row tiles of chunk
+// i).  Both tiles walk the same key tiles, so every K/V tile brought into
+// shared memory by TMA feeds two QK^T and two PV products.  The kept chunks of
+// row (h, i) are merged into runs of consecutive chunks once per CTA (a list in
+// shared memory; rows with more runs than it holds continue from the plan in
+// global memory), each run is cut into 128-key tiles, and the run holding the
+// diagonal is clipped at the last valid query row of the pair.  The first tile
+// of the pair stops at its own last row, so its tiles are a prefix of the
+// second's.
+//
+// Warp roles (320 threads; three warps share a sub-partition's 16K registers,
+// which caps a thread at 168 registers):
+//   warps 0-3   softmax + epilogue of query tile 0 (thread r = row r = TMEM lane r)
+//   warps 4-7   softmax + epilogue of query tile 1
+//   warp 8      TMA producer: both Q tiles once, K/V tiles into 2-stage rings
+//   warp 9      TMEM allocator and the single MMA-issuing thread
+// TMEM (512 columns): S_a at [128a, 128a+128); P_a (bf16, two per column) is
+// written over the first 64 columns of S_a and is the A operand of O_a += P_a V;
+// O_a at [256 + a*D, 256 + (a+1)*D).  Issue order per key tile t:
+//   PV_0(t), S_0(t+1), PV_1(t), S_1(t+1)
+// so while one warpgroup turns S into P the tensor core works for the other.
+// Online softmax in fp32, exp2 domain, one ex2.approx per element, lazy O
+// rescale (only when a warp's running max grows by more than 2^8).
+#include "common.cuh"
+#include "launchers.h"
+
+namespace dhsa {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kRangeCap = 1024;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct PairCfg {
+  static constexpr int kQSub = kBM * 128;   // one 64-column slice of a Q tile
+  static constexpr int kKVSub = kBN * 128;  // one 64-column slice of a K/V tile
+  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kKVBytes = kBN * D * 2;
+  static constexpr int kOffQ = 0;  // tile a at kOffQ + a * kQBytes
+  static constexpr int kOffK = 2 * kQBytes;
+  static constexpr int kOffV = kOffK + 2 * kKVBytes;
+  static constexpr int kOffRanges = kOffV + 2 * kKVBytes;
+  static constexpr int kOffBar = kOffRanges + kRangeCap * 8;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr uint32_t kColS = 0;    // + 128 a
+  static constexpr uint32_t kColO = 256;  // + D a
+  static_assert(256 + 2 * D <= 512, "TMEM budget");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+enum {
+  kBarQ = 0,
+  kBarKFull = 1,    // + stage
+  kBarKEmpty = 3,   // + stage
+  kBarVFull = 5,    // + stage
+  kBarVEmpty = 7,   // + stage
+  kBarSFull = 9,    // + query tile
+  kBarPFull = 11,   // + query tile
+  kBarOReady = 13,  // + query tile
+  kBarDrain = 15,
+  kNumBars = 16
+};
+
+// Key tiles of one work item: cached runs first, then (if the run list
+// overflowed) runs merged on the fly from the plan in global memory.
+struct TileWalk {
+  const int2* ranges;
+  int ncached, r;
+  const int* col;
+  const int* bounds;
+  int p, pend;
+  int k0, re, cap;
+  __device__ void init(const int2* ranges_, int ncached_, const int* col_, const int* bounds_, int resume,
+                       int p1, int cap_) {
+    ranges = ranges_;
+    ncached = ncached_;
+    r = 0;
+    col = col_;
+    bounds = bounds_;
+    p = resume;
+    pend = p1;
+    k0 = 0;
+    re = 0;
+    cap = cap_;
+  }
+  __device__ bool next(int& tk0, int& tke) {
+    if (k0 + kBN < re) {
+      k0 += kBN;
+    } else if (r < ncached) {
+      const int2 g = ranges[r++];
+      k0 = g.x;
+      re = min(g.y, cap);
+    } else {
+      if (p >= pend) return false;
+      int c = col[p++];
+      const int rs = bounds[c];
+      int e = bounds[c + 1];
+      while (p < pend && col[p] == c + 1) {
+        c = col[p++];
+        e = bounds[c + 1];
+      }
+      k0 = rs;
+      re = min(e, cap);
+    }
+    tk0 = k0;
+    tke = re;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// D(tmem) (+)= A(tmem) * B(smem desc), kind::f16.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attention_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+                          const int* __restrict__ bounds, const int* __restrict__ row_ptr,
+                          const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
+                          float scale_log2, uint32_t* status) {
+  using C = PairCfg<D>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto bar = [&](int idx) { return bar0 + 8u * static_cast<uint32_t>(idx); };
+  int2* ranges = reinterpret_cast<int2*>(smem + C::kOffRanges);
+  int* misc = reinterpret_cast<int*>(smem + C::kOffBar + 8 * kNumBars);
+  // misc[0] TMEM base, misc[1] abort flag, misc[2] cached runs, misc[3] resume position
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+  const int pair = blockIdx.x;
+  const int h = blockIdx.y;
+  const int ci = num_chunks - 1 - static_cast<int>(blockIdx.z);  // longest rows first
+  const int c_start = bounds[ci], c_end = bounds[ci + 1];
+  const int q0_0 = c_start + pair * 2 * kBM;
+  if (q0_0 >= c_end) return;  // uniform: this chunk has fewer tiles
+  const int q0_1 = q0_0 + kBM;
+  const bool valid1 = q0_1 < c_end;
+  const int q_end0 = min(q0_0 + kBM, c_end);
+  const int q_end1 = valid1 ? min(q0_1 + kBM, c_end) : q0_1;
+  const int cap = valid1 ? q_end1 : q_end0;
+  const int g = h / group;
+  const int row_id = h * num_chunks + ci;
+  const int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQ), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+      mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarPFull + s), kBM);
+      mbar_init(bar(kBarOReady + s), 1);
+    }
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp) {
+    // merge the row's kept chunks into runs of consecutive chunks
+    if (lane == 0) misc[3] = p1;
+    __syncwarp();
+    int nstart = 0, nend = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = p0; base < p1; base += 32) {
+      const int p = base + lane;
+      const bool valid = p < p1;
+      const int c = valid ? col[p] : 0;
+      int cprev = __shfl_up_sync(0xffffffffu, c, 1);
+      int cnext = __shfl_down_sync(0xffffffffu, c, 1);
+      if (lane == 0) cprev = (p > p0) ? col[p - 1] : -2;
+      if (lane == 31) cnext = (p + 1 < p1) ? col[p + 1] : -2;
+      const bool is_start = valid && (p == p0 || c != cprev + 1);
+      const bool is_end = valid && (p == p1 - 1 || cnext != c + 1);
+      const unsigned sm = __ballot_sync(0xffffffffu, is_start);
+      const unsigned em = __ballot_sync(0xffffffffu, is_end);
+      if (is_start) {
+        const int idx = nstart + __popc(sm & lt);
+        if (idx < kRangeCap) ranges[idx].x = bounds[c];
+        else if (idx == kRangeCap) misc[3] = p;
+      }
+      if (is_end) {
+        const int idx = nend + __popc(em & lt);
+        if (idx < kRangeCap) ranges[idx].y = bounds[c + 1];
+      }
+      nstart += __popc(sm);
+      nend += __popc(em);
+    }
+    if (lane == 0) misc[2] = min(nstart, kRangeCap);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(misc), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const int ncached = misc[2];
+  const int resume = misc[3];
+
+  // tile counts: all tiles (second query tile, or the only one) and the prefix of tile 0
+  int nt = 0, nt0 = 0;
+  {
+    TileWalk w;
+    w.init(ranges, ncached, col, bounds, resume, p1, cap);
+    int k0, ke;
+    while (w.next(k0, ke)) {
+      ++nt;
+      if (k0 < q_end0) ++nt0;
+    }
+  }
+  const int nt1 = valid1 ? nt : 0;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0 && nt > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(kBarQ), (valid1 ? 2 : 1) * C::kQBytes);
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a)
+        tma_load_3d(sbase + C::kOffQ + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h, q0_0);
+      if (valid1) {
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a)
+          tma_load_3d(sbase + C::kOffQ + C::kQBytes + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h, q0_1);
+      }
+      TileWalk w;
+      w.init(ranges, ncached, col, bounds, resume, p1, cap);
+      int k0, ke, issued = 0;
+      for (int t = 0; w.next(k0, ke); ++t) {
+        const int s = t & 1;
+        const uint32_t par = ((t >> 1) & 1) ^ 1;
+        if (!mbar_wait(bar(kBarKEmpty + s), par, abort_flag, status)) break;
+        mbar_arrive_expect_tx(bar(kBarKFull + s), C::kKVBytes);
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a)
+          tma_load_3d(sbase + C::kOffK + s * C::kKVBytes + a * C::kKVSub, &tm_k, bar(kBarKFull + s), a * 64, g, k0);
+        if (!mbar_wait(bar(kBarVEmpty + s), par, abort_flag, status)) {
+          issued = t + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(kBarVFull + s), C::kKVBytes);
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a)
+          tma_load_3d(sbase + C::kOffV + s * C::kKVBytes + a * C::kKVSub, &tm_v, bar(kBarVFull + s), a * 64, g, k0);
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA exits (bounded)
+        volatile int never = 0;
+        mbar_wait(bar(kBarQ), 0, &never, nullptr, 10000000ull);
+        for (int t = max(0, issued - 2); t < issued; ++t) {
+          mbar_wait(bar(kBarKFull + (t & 1)), (t >> 1) & 1, &never, nullptr, 10000000ull);
+          mbar_wait(bar(kBarVFull + (t & 1)), (t >> 1) & 1, &never, nullptr, 10000000ull);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 1);
+      const int nta[2] = {nt0, nt1};
+      auto issue_s = [&](int a, int t) {
+        const uint32_t qbase = sbase + C::kOffQ + a * C::kQBytes;
+        const uint32_t kbase = sbase + C::kOffK + (t & 1) * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(qbase + (kk >> 2) * C::kQSub + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * C::kKVSub + (kk & 3) * 32, 16, 1024);
+          umma_f16_ss(tmem + C::kColS + a * 128, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(kBarSFull + a));
+      };
+      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, status);
+      if (ok) ok = mbar_wait(bar(kBarKFull + 0), 0, abort_flag, status);
+      if (ok) {
+        tc_fence_after();
+        for (int a = 0; a < 2; ++a)
+          if (nta[a] > 0) issue_s(a, 0);
+        umma_commit(bar(kBarKEmpty + 0));
+      }
+      for (int t = 0; ok && t < nt; ++t) {
+        const int s = t & 1;
+        if (!mbar_wait(bar(kBarVFull + s), (t >> 1) & 1, abort_flag, status)) break;
+        const uint32_t vbase = sbase + C::kOffV + s * C::kKVBytes;
+        bool k_next_ready = false;
+        for (int a = 0; ok && a < 2; ++a) {
+          if (t >= nta[a]) continue;
+          if (!mbar_wait(bar(kBarPFull + a), t & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, C::kKVSub, 1024);
+            umma_f16_ts(tmem + C::kColO + a * D, tmem + C::kColS + a * 128 + kk * 8, bd, idesc_o,
+                        (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bar(kBarOReady + a));
+          if (t + 1 < nta[a]) {
+            if (!k_next_ready) {
+              if (!mbar_wait(bar(kBarKFull + ((t + 1) & 1)), ((t + 1) >> 1) & 1, abort_flag, status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(a, t + 1);
+          }
+        }
+        if (!ok) break;
+        umma_commit(bar(kBarVEmpty + s));
+        if (t + 1 < nt) umma_commit(bar(kBarKEmpty + ((t + 1) & 1)));
+      }
+      // every MMA issued above completes before TMEM is released
+      umma_commit(bar(kBarDrain));
+      volatile int never = 0;
+      mbar_wait(bar(kBarDrain), 0, &never, nullptr);
+    }
+  } else {
+    // ------------------------------------------------ softmax warpgroups
+    const int a = warp >> 2;  // query tile of this warpgroup
+    const int nta = a == 0 ? nt0 : nt1;
+    const int q0 = a == 0 ? q0_0 : q0_1;
+    const int q_end = a == 0 ? q_end0 : q_end1;
+    const int row = threadIdx.x & 127;
+    const int t_row = q0 + row;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::kColS + a * 128;
+    const uint32_t tO = tmem + lane_base + C::kColO + a * D;
+    float m_run = -INFINITY;  // running max of logits * scale * log2(e)
+    float l_run = 0.f;
+    TileWalk w;
+    w.init(ranges, ncached, col, bounds, resume, p1, cap);
+    int k0, ke;
+    bool ok = true;
+    for (int t = 0; t < nta && w.next(k0, ke); ++t) {
+      if (!mbar_wait(bar(kBarSFull + a), t & 1, abort_flag, status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kBN];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(tS + 0, r0);
+        tmem_ld32(tS + 32, r1);
+        tmem_ld32(tS + 64, r2);
+        tmem_ld32(tS + 96, r3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(r0[e]);
+          s[32 + e] = __uint_as_float(r1[e]);
+          s[64 + e] = __uint_as_float(r2[e]);
+          s[96 + e] = __uint_as_float(r3[e]);
+        }
+      }
+      if ((k0 + kBN > ke) || (k0 + kBN - 1 > q0)) {
+        const int lim = min(ke - k0, t_row - k0 + 1);  // valid columns: c < lim
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_tile = mx * scale_log2;
+      const bool any = __any_sync(0xffffffffu, m_tile > m_run + kRescaleLog2);
+      float alpha = 1.f;
+      if (any) {
+        const float m_new = fmaxf(m_run, m_tile);
+        alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
+        m_run = m_new;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float psum0 = 0.f, psum1 = 0.f;
+      uint32_t pk[kBN / 2];
+#pragma unroll
+      for (int c = 0; c < kBN; c += 2) {
+        const float e0 = ex2_approx(fmaf(s[c], scale_log2, -m_use));
+        const float e1 = ex2_approx(fmaf(s[c + 1], scale_log2, -m_use));
+        psum0 += e0;
+        psum1 += e1;
+        pk[c / 2] = pack_bf16(e0, e1);
+      }
+      l_run = l_run * alpha + (psum0 + psum1);
+      // P over the first 64 columns of S (the S values are already in registers)
+      tmem_st32p(tS + 0, pk);
+      tmem_st32p(tS + 32, pk + 32);
+      if (any && t > 0) {
+        // O is rescaled once PV(t-1) has landed
+        if (!mbar_wait(bar(kBarOReady + a), (t - 1) & 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + a));
+    }
+    if (ok && nta > 0 && mbar_wait(bar(kBarOReady + a), (nta - 1) & 1, abort_flag, status)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      const bool valid = t_row < q_end;
+      __nv_bfloat16* orow = out + (static_cast<size_t>(t_row) * num_q_heads + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 wv;
+            wv.x = pack_bf16(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+            wv.y = pack_bf16(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            wv.z = pack_bf16(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+            wv.w = pack_bf16(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + 32 * c + e) = wv;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int D>
+cudaError_t launch_attention_pair_dim(const AttnBf16Args& a, cudaStream_t stream) {
+  using C = PairCfg<D>;
+  CUtensorMap mq, mk, mv;
+  if (encode_qkv_map(&mq, a.q, a.num_q_heads, D, a.total_tokens, kBM) != CUDA_SUCCESS ||
+      encode_qkv_map(&mk, a.k, a.num_kv_heads, D, a.total_tokens, kBN) != CUDA_SUCCESS ||
+      encode_qkv_map(&mv, a.v, a.num_kv_heads, D, a.total_tokens, kBN) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  auto kern = attention_pair_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int pairs = (a.max_chunk_len + 2 * kBM - 1) / (2 * kBM);
+  dim3 grid(pairs, a.num_q_heads, a.num_chunks);
+  const float scale_log2 = a.scale * 1.4426950408889634f;
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
+                                                  a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
+                                                  a.num_q_heads / a.num_kv_heads, scale_log2, a.status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention_pair(const AttnBf16Args& a, cudaStream_t stream) {
+  if (a.head_dim == 128) return launch_attention_pair_dim<128>(a, stream);
+  if (a.head_dim == 64) return launch_attention_pair_dim<64>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dhsa

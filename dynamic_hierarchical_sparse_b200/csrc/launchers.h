@@ -60,6 +60,10 @@ struct AttnBf16Args {
   uint32_t* status;
 };
 cudaError_t launch_attention_bf16(const AttnBf16Args& a, cudaStream_t stream);
+// head_dim 64 / 128: two query tiles per CTA, P kept in TMEM.
+cudaError_t launch_attention_pair(const AttnBf16Args& a, cudaStream_t stream);
+// TMA view of a packed THD bf16 tensor (see attention_bf16.cu).
+CUresult encode_qkv_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows);
 
 // Diagnostic: a kernel whose only wait can never be satisfied, bounded by limit_ns.
 cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);

@@ -75,3 +75,30 @@ def test_workload_full_size(spec):
     print(spec.name, "sampled rows:", len(sample), "max_err=%.3g max|O|=%.3g median|O|=%.3g"
           % (err.max(), np.abs(want).max(), np.median(np.abs(want))))
     assert err.max() <= tol
+
+
+def test_select_microbench_rows():
+    """The select micro-benchmark's configuration (n ~ 3200 chunks, 32 heads,
+    keep 5 %): sampled rows of the GPU plan equal the oracle's selection from
+    the same fp32 scores (integer work: bit-exact)."""
+    import bench
+
+    cu, bounds, sptr = bench.select_micro_inputs(0)
+    spec = bench.SELECT_MICRO
+    dev = torch.device("cuda")
+    prob = api.Problem(cu, bounds, sptr, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, torch.bfloat16, dev)
+    n = prob.num_chunks
+    gen = torch.Generator(device=dev).manual_seed(0)
+    scores = torch.randn(spec.num_q_heads, n, n, generator=gen, device=dev, dtype=torch.float32)
+    plan = api.topk_select(scores, prob, spec.budget, check=True)
+    rows = gpu_rows(plan, spec.num_q_heads * n)
+    rng = np.random.default_rng(3)
+    b = spec.budget
+    for r in list(rng.choice(spec.num_q_heads * n, size=300, replace=False)) + [n - 1, spec.num_q_heads * n - 1]:
+        h, i = int(r) // n, int(r) % n
+        S = scores[h, i, :i].double().cpu().numpy()
+        keep = O.row_budget(i, b.kind, b.k, b.num, b.den)
+        want = sorted(O.select_row(list(S), list(range(i)), keep)) + [i]
+        assert rows[r] == want, (h, i)
+    del scores
+    torch.cuda.empty_cache()
