@@ -6,7 +6,7 @@
 
 #include <mutex>
 
-#include "../../include/dhsa.h"
+#include "dhsa.h"
 #include "common.cuh"
 #include "launchers.h"
 

@@ -19,12 +19,16 @@
 // of the pair stops at its own last row, so its tiles are a prefix of the
 // second's.
 //
-// Warp roles (320 threads; three warps share a sub-partition's 16K registers,
-// which caps a thread at 168 registers):
+// Warp roles (384 threads = three warpgroups):
 //   warps 0-3   softmax + epilogue of query tile 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of query tile 1
 //   warp 8      TMA producer: both Q tiles once, K/V tiles into 2-stage rings
 //   warp 9      TMEM allocator and the single MMA-issuing thread
+//   warps 10-11 idle
+// The launch gives every thread 168 registers (three warps share a
+// sub-partition's 16K); the third warpgroup then hands registers back
+// (setmaxnreg.dec to 56) and the softmax warpgroups take them (224), enough to
+// hold a whole 128-column row of S without spilling.
 // TMEM (512 columns): S_a at [128a, 128a+128); P_a (bf16, two per column) is
 // written over the first 64 columns of S_a and is the A operand of O_a += P_a V;
 // O_a at [256 + a*D, 256 + (a+1)*D).  Issue order per key tile t:
@@ -33,6 +37,7 @@
 // Online softmax in fp32, exp2 domain, one ex2.approx per element, lazy O
 // rescale (only when a warp's running max grows by more than 2^8).
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "launchers.h"
 
 namespace dhsa {
@@ -40,7 +45,15 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsSoftmax = 224;  // 8 warps x 224 + 4 warps x 56 = 384 x 168
+constexpr uint32_t kRegsOther = 56;
+// Every kPolyPairEvery-th pair of softmax columns takes its exp2 on the FMA
+// pipe (exp2_fma) instead of the MUFU unit; 0 keeps every exp2 on MUFU.
+constexpr int kPolyPairEvery = 0;
+// Two exponentials per MUFU operation (ex2.approx.f16x2): the arguments are
+// rounded to fp16 (11-bit significand), finer than the bf16 the results feed.
+constexpr bool kExpHalf2 = false;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -87,7 +100,7 @@ struct TileWalk {
   const int* bounds;
   int p, pend;
   int k0, re, cap;
-  __device__ void init(const int2* ranges_, int ncached_, const int* col_, const int* bounds_, int resume,
+  __device__ __forceinline__ void init(const int2* ranges_, int ncached_, const int* col_, const int* bounds_, int resume,
                        int p1, int cap_) {
     ranges = ranges_;
     ncached = ncached_;
@@ -100,7 +113,7 @@ struct TileWalk {
     re = 0;
     cap = cap_;
   }
-  __device__ bool next(int& tk0, int& tke) {
+  __device__ __forceinline__ bool next(int& tk0, int& tke) {
     if (k0 + kBN < re) {
       k0 += kBN;
     } else if (r < ncached) {
@@ -128,6 +141,30 @@ struct TileWalk {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// exp2 of two fp32 arguments through one ex2.approx.f16x2; results widened to fp32.
+__device__ __forceinline__ float2 ex2_pair_f16(float x0, float x1) {
+  uint32_t h;
+  asm("{\n\t.reg .b32 t;\n\t"
+      "cvt.rn.f16x2.f32 t, %2, %1;\n\t"
+      "ex2.approx.f16x2 %0, t;\n\t}"
+      : "=r"(h)
+      : "f"(x0), "f"(x1));
+  float2 r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t"
+      "cvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(h));
+  return r;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -253,6 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int nt1 = valid1 ? nt : 0;
 
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
   if (warp == kProducerWarp) {
     if (lane == 0 && nt > 0) {
       tma_prefetch_desc(&tm_q);
@@ -302,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && nt > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 1);
-      const int nta[2] = {nt0, nt1};
       auto issue_s = [&](int a, int t) {
         const uint32_t qbase = sbase + C::kOffQ + a * C::kQBytes;
         const uint32_t kbase = sbase + C::kOffK + (t & 1) * C::kKVBytes;
@@ -319,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         for (int a = 0; a < 2; ++a)
-          if (nta[a] > 0) issue_s(a, 0);
+          if ((a == 0 ? nt0 : nt1) > 0) issue_s(a, 0);
         umma_commit(bar(kBarKEmpty + 0));
       }
       for (int t = 0; ok && t < nt; ++t) {
@@ -328,7 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vbase = sbase + C::kOffV + s * C::kKVBytes;
         bool k_next_ready = false;
         for (int a = 0; ok && a < 2; ++a) {
-          if (t >= nta[a]) continue;
+          const int nta = a == 0 ? nt0 : nt1;
+          if (t >= nta) continue;
           if (!mbar_wait(bar(kBarPFull + a), t & 1, abort_flag, status)) {
             ok = false;
             break;
@@ -341,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (t > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(bar(kBarOReady + a));
-          if (t + 1 < nta[a]) {
+          if (t + 1 < nta) {
             if (!k_next_ready) {
               if (!mbar_wait(bar(kBarKFull + ((t + 1) & 1)), ((t + 1) >> 1) & 1, abort_flag, status)) {
                 ok = false;
@@ -362,7 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(bar(kBarDrain), 0, &never, nullptr);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------ softmax warpgroups
     const int a = warp >> 2;  // query tile of this warpgroup
     const int nta = a == 0 ? nt0 : nt1;
@@ -385,32 +426,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      // S row -> registers in two halves: the second half is still loading
+      // while the first half is masked and max-reduced.
       float s[kBN];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tS + 0, r0);
-        tmem_ld32(tS + 32, r1);
-        tmem_ld32(tS + 64, r2);
-        tmem_ld32(tS + 96, r3);
-        tmem_wait_ld();
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const bool masked = (k0 + kBN > ke) || (k0 + kBN - 1 > q0);
+      const int lim = min(ke - k0, t_row - k0 + 1);  // valid columns: c < lim
+      auto take_half = [&](int base, uint32_t (&ra)[32], uint32_t (&rb)[32]) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          s[e] = __uint_as_float(r0[e]);
-          s[32 + e] = __uint_as_float(r1[e]);
-          s[64 + e] = __uint_as_float(r2[e]);
-          s[96 + e] = __uint_as_float(r3[e]);
+          s[base + e] = __uint_as_float(ra[e]);
+          s[base + 32 + e] = __uint_as_float(rb[e]);
         }
-      }
-      if ((k0 + kBN > ke) || (k0 + kBN - 1 > q0)) {
-        const int lim = min(ke - k0, t_row - k0 + 1);  // valid columns: c < lim
+        if (masked) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c >= lim) s[c] = -INFINITY;
-      }
-      float mx = s[0];
+          for (int c = base; c < base + kBN / 2; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        // row max as a tree of 3-input maxima (short dependency chains)
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_tile = mx * scale_log2;
+        for (int c = base; c < base + kBN / 2; c += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mp[q] = fmax3(mp[q], s[c + q], s[c + 4 + q]);
+        }
+      };
+      {
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        tmem_ld32(tS + 0, ra);
+        tmem_ld32(tS + 32, rb);
+        tmem_wait_ld();
+        reg_dep32(ra);
+        reg_dep32(rb);
+        tmem_ld32(tS + 64, rc);
+        tmem_ld32(tS + 96, rd);
+        take_half(0, ra, rb);
+        tmem_wait_ld();
+        reg_dep32(rc);
+        reg_dep32(rd);
+        take_half(kBN / 2, rc, rd);
+      }
+      const float m_tile = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * scale_log2;
       const bool any = __any_sync(0xffffffffu, m_tile > m_run + kRescaleLog2);
       float alpha = 1.f;
       if (any) {
@@ -419,17 +474,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float psum0 = 0.f, psum1 = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[kBN / 2];
 #pragma unroll
       for (int c = 0; c < kBN; c += 2) {
-        const float e0 = ex2_approx(fmaf(s[c], scale_log2, -m_use));
-        const float e1 = ex2_approx(fmaf(s[c + 1], scale_log2, -m_use));
-        psum0 += e0;
-        psum1 += e1;
+        const float x0 = fmaf(s[c], scale_log2, -m_use);
+        const float x1 = fmaf(s[c + 1], scale_log2, -m_use);
+        float e0, e1;
+        if (kExpHalf2) {
+          const float2 e = ex2_pair_f16(x0, x1);
+          e0 = e.x;
+          e1 = e.y;
+        } else if (kPolyPairEvery > 0 && (c / 2) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
+          e0 = exp2_fma(x0);
+          e1 = exp2_fma(x1);
+        } else {
+          e0 = ex2_approx(x0);
+          e1 = ex2_approx(x1);
+        }
+        ps[(c / 2) & 3] += e0 + e1;
         pk[c / 2] = pack_bf16(e0, e1);
       }
-      l_run = l_run * alpha + (psum0 + psum1);
+      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       // P over the first 64 columns of S (the S values are already in registers)
       tmem_st32p(tS + 0, pk);
       tmem_st32p(tS + 32, pk + 32);
@@ -445,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[32];
           tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
+          reg_dep32(o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(tO + 32 * c, o);
@@ -464,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
         tmem_wait_ld();
+        reg_dep32(o);
         if (valid) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
