@@ -39,9 +39,11 @@ METRIC = "DHSA prefill tokens/s at 128K (1 B200); attn tensor-pipe % of peak on 
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = W.LLAMA_128K.name
 
-# ncu (gpu__time_duration / dram__bytes) figures for the attention kernel at the
-# default workload; None until a capture of the current kernel exists.
-ATTN_TRAFFIC_BYTES_PER_LAUNCH = None
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention_pair_kernel<128>
+# launch at the default 128K workload (9.45 GB + 1.16 GB), from a one-pass ncu
+# capture of the current kernel (profiles/attention_pair_llama128k_dram.md).
+# Must be reset to None whenever that kernel changes.
+ATTN_TRAFFIC_BYTES_PER_LAUNCH = 10.61e9
 
 
 def _peaks():
@@ -318,10 +320,12 @@ def bench_gpu(args):
         "t_plan_ms": t_plan * 1e3, "t_attn_ms": t_attn * 1e3,
         "plan_hbm_gbs": reduce_bytes / t_plan / 1e9,
         "roofline": {
-            "kernel": "attention_bf16_kernel<128,128>", "bound": "tensor", "achieved": achieved_tflops,
+            "kernel": "attention_pair_kernel<%d>" % spec.head_dim if spec.head_dim in (64, 128)
+                      else "attention_bf16_kernel<%d,64>" % spec.head_dim,
+            "bound": "tensor", "achieved": achieved_tflops,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved_tflops / peak,
             "peak_kind": "%s bf16 dense, sustained (kernel timed inside a seconds-long loop)" % peaks["source"],
-            "traffic": ATTN_TRAFFIC_BYTES_PER_LAUNCH,
+            "traffic": ATTN_TRAFFIC_BYTES_PER_LAUNCH if spec.name == DEFAULT_WORKLOAD else None,
             "algorithmic_flops_per_launch": flops_attn,
         },
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

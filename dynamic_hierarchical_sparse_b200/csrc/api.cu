@@ -15,7 +15,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
-constexpr int kMaxSelectCandidates = 12000;  // per-row staging in shared memory
+constexpr int kMaxSelectCandidates = 48000;  // per-row staging in shared memory (192 KB)
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 

@@ -184,3 +184,45 @@ def test_product_package_does_not_import_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 with open(os.path.join(dirpath, fn)) as f:
                     assert not pat.search(f.read()), fn
+
+
+def _floor_sum(n, m, a, c):
+    """The select kernel's lattice-point recursion, restated (Python ints)."""
+    total = 0
+    while n > 0:
+        if a >= m:
+            total += (n * (n - 1) // 2) * (a // m)
+            a %= m
+        if c >= m:
+            total += n * (c // m)
+            c %= m
+        y = a * n + c
+        if y < m:
+            break
+        n, c, m, a = y // m, y % m, a, m
+    return total
+
+
+def _plan_entries(L, budget):
+    if L <= 0:
+        return 0
+    if budget.kind == W.BUDGET_TOPK:
+        k = budget.k
+        s = L * (L - 1) // 2 if L <= k else k * (k - 1) // 2 + k * (L - k)
+    elif budget.num >= budget.den:
+        s = L * (L - 1) // 2
+    else:
+        s = _floor_sum(L, budget.den, budget.num, budget.den - 1)
+    return s + L
+
+
+@pytest.mark.parametrize("budget", [W.Budget.topk(0), W.Budget.topk(1), W.Budget.topk(7),
+                                    W.Budget.fraction(1, 20), W.Budget.fraction(1, 10),
+                                    W.Budget.fraction(3, 7), W.Budget.fraction(5, 4), W.Budget.fraction(0, 3)])
+def test_closed_form_plan_offsets(budget):
+    """Closed form of the per-chunk plan offsets used by the select kernel
+    equals the running sum of (row budget + 1) from the oracle's rule."""
+    running = 0
+    for L in range(0, 3000):
+        assert _plan_entries(L, budget) == running, L
+        running += O.row_budget(L, budget.kind, budget.k, budget.num, budget.den) + 1
