@@ -148,13 +148,20 @@ def _barrier(world):
         dist.barrier()
 
 
-def _max_over_ranks(x: float, world: int) -> float:
+def _max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Largest value over all ranks (the timed span of the slowest replica)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_replica: int, steps: int, max_elapsed_s: float) -> float:
+    """Weak scaling: every rank runs one replica of the workload; the job's rate is
+    all ranks' tokens over the slowest rank's timed span."""
+    return world * tokens_per_replica * steps / max_elapsed_s
 
 
 def run_cpu_oracle(inp, budget_seconds: float = 20.0):
@@ -268,7 +275,7 @@ def bench_gpu(args):
     if planner.status() != 0 or attn.status() != 0:
         raise RuntimeError("device-side status set during the timed region")
     max_elapsed = _max_over_ranks(elapsed_s, world)
-    value = world * T * args.steps / max_elapsed
+    value = whole_job_tokens_per_s(world, T, args.steps, max_elapsed)
 
     # ---------------- end to end through the public API with host buffers
     hq = inp.q.pin_memory()
@@ -295,7 +302,7 @@ def bench_gpu(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_s = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-    e2e_value = world * T * e2e_steps / e2e_s
+    e2e_value = whole_job_tokens_per_s(world, T, e2e_steps, e2e_s)
     h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
     d2h = hout.numel() * hout.element_size()
 
