@@ -15,7 +15,6 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
-constexpr int kMaxSelectCandidates = 48000;  // per-row staging in shared memory (192 KB)
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -65,15 +64,6 @@ dhsa_status check_problem(const dhsa_problem* p) {
   return DHSA_OK;
 }
 
-int max_chunks_per_seq(const dhsa_problem* p) {
-  int m = 0;
-  for (int b = 0; b < p->num_seqs; ++b) {
-    const int c = p->h_seq_chunk_ptr[b + 1] - p->h_seq_chunk_ptr[b];
-    if (c > m) m = c;
-  }
-  return m;
-}
-
 int max_chunk_len(const dhsa_problem* p) {
   int m = 0;
   for (int c = 0; c < p->num_chunks; ++c) {
@@ -113,11 +103,9 @@ BudgetArgs to_args(const dhsa_budget& b) { return BudgetArgs{b.kind, b.k, b.num,
 // Selection core shared by dhsa_topk_select and dhsa_plan (after validation).
 dhsa_status run_select(const float* scores, const dhsa_problem* p, const dhsa_budget& budget, int32_t* row_ptr,
                        int32_t* col, uint32_t* status, cudaStream_t stream) {
-  const int cap = max_chunks_per_seq(p) > 1 ? max_chunks_per_seq(p) - 1 : 1;
-  if (cap > kMaxSelectCandidates) return DHSA_ERR_UNSUPPORTED;
   const int64_t per_head = nnz_per_head(p, budget);
   return cuda_status(launch_topk_select(scores, p->num_chunks, p->num_q_heads, p->seq_chunk_ptr, p->num_seqs,
-                                        to_args(budget), row_ptr, col, static_cast<int>(per_head), cap, status,
+                                        to_args(budget), row_ptr, col, static_cast<int>(per_head), status,
                                         stream));
 }
 

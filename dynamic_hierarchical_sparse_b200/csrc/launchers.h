@@ -26,13 +26,11 @@ cudaError_t launch_chunk_similarity(const float* qc, const float* kc, int num_q_
                                     int num_chunks, int head_dim, const int* seq_chunk_ptr,
                                     int num_seqs, float* scores, cudaStream_t stream);
 
-// Step 3.  key_capacity >= the largest number of admissible candidates of any
-// row (chunks per sequence - 1).
-size_t topk_select_smem_bytes(int key_capacity);
+// Step 3 (any number of candidates per row).
 cudaError_t launch_topk_select(const float* scores, int num_chunks, int num_q_heads,
                                const int* seq_chunk_ptr, int num_seqs, BudgetArgs budget,
-                               int* row_ptr, int* col, int nnz_per_head, int key_capacity,
-                               uint32_t* status, cudaStream_t stream);
+                               int* row_ptr, int* col, int nnz_per_head, uint32_t* status,
+                               cudaStream_t stream);
 
 // Step 4, fp32.
 cudaError_t launch_attention_f32(const float* q, const float* k, const float* v, const int* bounds,

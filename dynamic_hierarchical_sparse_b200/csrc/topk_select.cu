@@ -10,51 +10,80 @@
 // chunks j < i of the same sequence with the largest S[h, i, j] (ties to the
 // lower j), plus the diagonal chunk i, written in ascending order.
 //
-// One 256-thread CTA per row.  The row's scores are read once (coalesced) into
-// shared memory as order-preserving 32-bit keys, the first digit histogram
-// being built during that load; an MSB-first radix select (8-bit digits over a
-// block-shared 256-bin histogram) finds the k-th largest key exactly, stopping
-// early once the threshold bucket is taken whole.  Compaction is in index
-// order: each warp owns a contiguous segment, per-warp counts of keys above and
-// equal to the threshold give every warp its output offset and its share of
-// the equal keys (lowest index first), and ballots place the keys.  The row's
-// plan offset comes in closed form (plan_entries), not from a loop over the
-// earlier chunks.
+// One warp per row, eight consecutive rows (chunks i) of one query head per
+// CTA.  Row offsets in the CSR follow from one closed-form offset per CTA
+// (plan_entries) plus the budgets of the CTA's earlier rows.
+//
+// Rows of at most kSurvCap candidates are staged whole in the warp's shared
+// memory as order-preserving 32-bit keys.  Longer rows with a budget of at
+// most 1/8 of the row first try a filter: the warp sorts 64 evenly spaced
+// samples and takes as threshold tau the sample a few ranks below the
+// budget's quantile; one coalesced sweep keeps the keys >= tau ("survivors",
+// in index order).  When at least `keep` keys survive and they fit, the k-th
+// largest key is among them and the exact selection runs on them only;
+// otherwise (an unlucky sample, heavy ties, large budgets) the warp selects
+// from the row in global memory directly, so the result never depends on the
+// sample and no row is too long.  Either way an MSB-first radix select (8-bit
+// digits over a warp-private 256-bin histogram) finds the k-th largest key
+// exactly, stopping early once the threshold bucket is taken whole, and one
+// pass in index order writes the keys above it plus the lowest-indexed keys
+// equal to it.
 #include "common.cuh"
 #include "launchers.h"
 
 namespace dhsa {
 namespace {
 
-constexpr int kSelThreads = 256;
-constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelWarps = 8;  // rows per CTA
+constexpr int kSelThreads = 32 * kSelWarps;
+constexpr int kSurvCap = 896;           // staged keys per warp
+constexpr int kFilterMaxCandidates = 65535;  // survivor indices are 16-bit
+constexpr int kSamples = 64;
+constexpr int kSampleMargin = 5;  // ranks below the budget's sample quantile
+constexpr int kBatch = 16;        // loads in flight per lane in the sweeps
+
+struct WarpScratch {
+  int hist[256];
+  uint32_t key[kSurvCap];
+  uint16_t idx[kSurvCap];
+};
+
+// a / b and a % b on non-negative 64-bit values, in 32-bit arithmetic when both fit
+__device__ __forceinline__ unsigned long long udiv(unsigned long long a, unsigned long long b) {
+  if (((a | b) >> 32) == 0) return static_cast<uint32_t>(a) / static_cast<uint32_t>(b);
+  return a / b;
+}
 
 __device__ __forceinline__ int row_budget(int i_local, const BudgetArgs& b) {
   if (b.kind == 0) return min(b.k, i_local);
-  // ceil(i_local * num / den), capped at i_local (64-bit to avoid overflow)
-  const long long want = (static_cast<long long>(i_local) * b.num + b.den - 1) / b.den;
-  return static_cast<int>(min(static_cast<long long>(i_local), want));
+  // ceil(i_local * num / den), capped at i_local
+  const unsigned long long want =
+      udiv(static_cast<unsigned long long>(i_local) * b.num + b.den - 1, static_cast<unsigned long long>(b.den));
+  return static_cast<int>(min(static_cast<unsigned long long>(i_local), want));
 }
 
 // sum_{l=0}^{n-1} floor((a*l + c) / m) for n, a, c >= 0 and m >= 1: lattice
 // points under a line, counted by the Euclid-like reduction (swap the roles of
 // a and m after taking out the integer parts), O(log) steps.
-__device__ long long floor_sum(long long n, long long m, long long a, long long c) {
-  long long total = 0;
+__device__ unsigned long long floor_sum(unsigned long long n, unsigned long long m, unsigned long long a,
+                                        unsigned long long c) {
+  unsigned long long total = 0;
   while (n > 0) {
     if (a >= m) {
-      total += (n * (n - 1) / 2) * (a / m);
-      a %= m;
+      const unsigned long long q = udiv(a, m);
+      total += (n * (n - 1) / 2) * q;
+      a -= q * m;
     }
     if (c >= m) {
-      total += n * (c / m);
-      c %= m;
+      const unsigned long long q = udiv(c, m);
+      total += n * q;
+      c -= q * m;
     }
-    const long long y_max = a * n + c;
+    const unsigned long long y_max = a * n + c;
     if (y_max < m) break;
-    n = y_max / m;
-    c = y_max % m;
-    const long long t = m;
+    n = udiv(y_max, m);
+    c = y_max - n * m;
+    const unsigned long long t = m;
     m = a;
     a = t;
   }
@@ -72,7 +101,7 @@ __device__ long long plan_entries(long long L, const BudgetArgs& b) {
   } else if (b.num >= b.den) {
     s = L * (L - 1) / 2;  // ceil(l * num / den) >= l: every earlier chunk
   } else {
-    s = floor_sum(L, b.den, b.num, b.den - 1);  // sum of ceil(l * num / den)
+    s = static_cast<long long>(floor_sum(L, b.den, b.num, b.den - 1));  // sum of ceil(l * num / den)
   }
   return s + L;
 }
@@ -81,6 +110,11 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s);
   if (u == 0x80000000u) u = 0u;  // -0 ranks equal to +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// the float whose order key is k (+0 for the key of both zeros)
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 __device__ __forceinline__ int seq_of_chunk(const int* __restrict__ ptr, int num_seqs, int c) {
@@ -92,185 +126,250 @@ __device__ __forceinline__ int seq_of_chunk(const int* __restrict__ ptr, int num
   return lo;
 }
 
-// grid: x = chunk i, y = query head; one 256-thread CTA per row (h, i).
-__global__ void __launch_bounds__(kSelThreads)
-    topk_select_kernel(const float* __restrict__ scores, int num_chunks, int num_q_heads,
-                       const int* __restrict__ seq_chunk_ptr, int num_seqs, BudgetArgs budget,
-                       int* __restrict__ row_ptr, int* __restrict__ col, int nnz_per_head,
-                       int key_capacity, uint32_t* status) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ int hist[256];
-  __shared__ int s_gt[kSelWarps], s_eq[kSelWarps];
-  __shared__ int s_prefix, s_digit, s_above, s_count;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);
-  const int i = blockIdx.x, h = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  // plan offset of chunk i within one head: entries of every earlier chunk
-  if (tid == 0) {
-    long long acc = 0;
-    for (int b = 0; b < num_seqs; ++b) {
-      const int c0 = seq_chunk_ptr[b];
-      if (c0 >= i) break;
-      acc += plan_entries(min(seq_chunk_ptr[b + 1], i) - c0, budget);
+// Sorts 64 keys held two per lane (element e = slot * 32 + lane) into
+// descending order with a bitonic network.
+__device__ __forceinline__ void bitonic64_desc(uint32_t& v0, uint32_t& v1, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {
+        const uint32_t hi = max(v0, v1), lo = min(v0, v1);
+        v0 = hi;
+        v1 = lo;
+      } else {
+        const uint32_t p0 = __shfl_xor_sync(0xffffffffu, v0, j);
+        const uint32_t p1 = __shfl_xor_sync(0xffffffffu, v1, j);
+        const bool low = (lane & j) == 0;
+        // a block of size k sorts descending when (e & k) == 0
+        const bool d0 = (lane & k) == 0;
+        const bool d1 = k == 32 ? false : (lane & k) == 0;
+        v0 = (d0 == low) ? max(v0, p0) : min(v0, p0);
+        v1 = (d1 == low) ? max(v1, p1) : min(v1, p1);
+      }
     }
-    s_prefix = static_cast<int>(acc);
   }
-  for (int q = tid; q < 256; q += kSelThreads) hist[q] = 0;
-  __syncthreads();
-  const int prefix = s_prefix;
+}
 
-  const int b = seq_of_chunk(seq_chunk_ptr, num_seqs, i);
-  const int c0 = seq_chunk_ptr[b];
-  const int m = i - c0;  // admissible candidates c0 .. i-1
-  const int keep = row_budget(m, budget);
-  const int row = h * num_chunks + i;
-  const int off = h * nnz_per_head + prefix;
-  if (tid == 0) {
-    row_ptr[row] = off;
-    if (row == num_q_heads * num_chunks - 1) row_ptr[row + 1] = off + keep + 1;
-  }
-  int* out = col + off;
-  if (keep >= m) {  // every admissible chunk is kept
-    for (int j = tid; j < m; j += kSelThreads) out[j] = c0 + j;
-    if (tid == 0) out[m] = i;
-    return;
-  }
-  if (keep == 0) {
-    if (tid == 0) out[0] = i;
-    return;
-  }
-  if (m > key_capacity) {  // host sizing guarantees this cannot happen
-    if (tid == 0) report(status, kDevCheck);
-    return;
-  }
-
-  // load the row once (coalesced) as order-preserving keys; first digit pass fused in
-  const float* srow = scores + (static_cast<size_t>(h) * num_chunks + i) * num_chunks + c0;
-#pragma unroll 4
-  for (int j = tid; j < m; j += kSelThreads) {
-    const uint32_t kj = order_key(__ldcs(srow + j));
-    keys[j] = kj;
-    atomicAdd(&hist[kj >> 24], 1);
-  }
-  __syncthreads();
-
-  uint32_t prefix_bits = 0, prefix_mask = 0;
-  int remaining = keep;  // still to take among keys matching prefix_bits under prefix_mask
+// Exact selection of the `keep` largest of n keys (ties to the lower index),
+// written ascending by index to out[0..keep).  Keys come from get_key(t),
+// their chunk ids from get_col(t), t ascending = index ascending.  hist[] holds
+// the first digit's counts when first_done, else it is zero on entry.
+template <typename GetKey, typename GetCol>
+__device__ __forceinline__ bool warp_select(int n, int keep, int* hist, bool first_done, GetKey get_key,
+                                            GetCol get_col, int* __restrict__ out, int lane) {
+  uint32_t bits = 0, mask = 0;
+  int remaining = keep;  // still to take among keys matching bits under mask
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    if (pass > 0) {
-      for (int j = tid; j < m; j += kSelThreads) {
-        const uint32_t kj = keys[j];
-        if ((kj & prefix_mask) == prefix_bits) atomicAdd(&hist[(kj >> shift) & 255u], 1);
+    if (pass > 0 || !first_done) {
+      if (pass > 0) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) hist[32 * q + lane] = 0;
+        __syncwarp();
       }
-      __syncthreads();
+      for (int t = lane; t < n; t += 32) {
+        const uint32_t k = get_key(t);
+        if ((k & mask) == bits) atomicAdd(&hist[(k >> shift) & 255u], 1);
+      }
+      __syncwarp();
     }
-    if (warp == 0) {
-      // lane L owns digits 255-8L down to 248-8L (descending order across lanes)
-      int cnt[8];
-      int mine = 0;
+    // lane L owns digits 255-8L down to 248-8L (descending order across lanes)
+    int cnt[8];
+    int mine = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      cnt[q] = hist[255 - 8 * lane - q];
+      mine += cnt[q];
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - mine;
+    const bool here = excl < remaining && remaining <= incl;
+    int digit = 0, above = 0, count = 0;
+    if (here) {
+      int run = excl;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        cnt[q] = hist[255 - 8 * lane - q];
-        mine += cnt[q];
-      }
-      int incl = mine;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int excl = incl - mine;
-      if (excl < remaining && remaining <= incl) {
-        int run = excl;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (run + cnt[q] >= remaining) {
-            s_digit = 255 - 8 * lane - q;
-            s_above = run;
-            s_count = cnt[q];
-            break;
-          }
-          run += cnt[q];
+        if (run + cnt[q] >= remaining) {
+          digit = 255 - 8 * lane - q;
+          above = run;
+          count = cnt[q];
+          break;
         }
+        run += cnt[q];
       }
     }
-    __syncthreads();
-    const int digit = s_digit, above = s_above, count = s_count;
+    const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    count = __shfl_sync(0xffffffffu, count, src);
+    __syncwarp();
     remaining -= above;
-    prefix_bits |= static_cast<uint32_t>(digit) << shift;
-    prefix_mask |= 0xFFu << shift;
+    bits |= static_cast<uint32_t>(digit) << shift;
+    mask |= 0xFFu << shift;
     if (remaining == count) break;  // the whole bucket is taken: no finer digits needed
-    for (int q = tid; q < 256; q += kSelThreads) hist[q] = 0;
-    __syncthreads();
   }
-  // selected: (key & mask) > prefix, plus the lowest-indexed `need_eq` keys with
-  // (key & mask) == prefix (all of them when the bucket was taken whole)
-  const uint32_t thr = prefix_bits, msk = prefix_mask;
-  const int need_eq = remaining;
-
-  // compaction in index order: warp w owns the contiguous segment [lo, hi)
-  const int seg = (m + kSelWarps - 1) / kSelWarps;
-  const int lo = min(m, warp * seg), hi = min(m, lo + seg);
-  int n_gt = 0, n_eq = 0;
-  for (int base = lo; base < hi; base += 32) {
-    const int j = base + lane;
-    const uint32_t kj = j < hi ? (keys[j] & msk) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, j < hi && kj > thr));
-    n_eq += __popc(__ballot_sync(0xffffffffu, j < hi && kj == thr));
-  }
-  if (lane == 0) {
-    s_gt[warp] = n_gt;
-    s_eq[warp] = n_eq;
-  }
-  __syncthreads();
-  int eq_before = 0, sel_before = 0;
-  for (int w = 0; w < warp; ++w) {
-    const int eqb = eq_before;
-    eq_before += s_eq[w];
-    sel_before += s_gt[w] + min(max(need_eq - eqb, 0), s_eq[w]);
-  }
-  int written = sel_before, eq_seen = eq_before;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += 32) {
-    const int j = base + lane;
-    const uint32_t kj = j < hi ? (keys[j] & msk) : 0u;
-    const bool gt = j < hi && kj > thr;
-    const bool eq = j < hi && kj == thr;
+  // selected: (key & mask) > bits, plus the lowest-indexed `remaining` keys with
+  // (key & mask) == bits (all of them when the bucket was taken whole)
+  const unsigned lt = (1u << lane) - 1u;
+  int written = 0, eq_seen = 0;
+  for (int base = 0; base < n && written < keep; base += 32) {
+    const int t = base + lane;
+    const uint32_t k = t < n ? (get_key(t) & mask) : 0u;
+    const bool gt = t < n && k > bits;
+    const bool eq = t < n && k == bits;
     const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const bool sel = gt || (eq && (eq_seen + __popc(eqm & lt_mask)) < need_eq);
+    const bool sel = gt || (eq && (eq_seen + __popc(eqm & lt)) < remaining);
     const unsigned selm = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[written + __popc(selm & lt_mask)] = c0 + j;
+    if (sel) out[written + __popc(selm & lt)] = get_col(t);
     written += __popc(selm);
     eq_seen += __popc(eqm);
   }
-  if (warp == kSelWarps - 1 && lane == 0) {
-    out[keep] = i;
-    if (written != keep) report(status, kDevCheck);
+  return written == keep;
+}
+
+// grid: x = group of kSelWarps consecutive chunks, y = query head.
+__global__ void __launch_bounds__(kSelThreads)
+    topk_select_kernel(const float* __restrict__ scores, int num_chunks, int num_q_heads,
+                       const int* __restrict__ seq_chunk_ptr, int num_seqs, BudgetArgs budget,
+                       int* __restrict__ row_ptr, int* __restrict__ col, int nnz_per_head, uint32_t* status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ int s_entries[kSelWarps];
+  __shared__ long long s_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int i0 = blockIdx.x * kSelWarps;
+  const int i = i0 + warp;
+  const bool valid = i < num_chunks;
+  WarpScratch& ws = reinterpret_cast<WarpScratch*>(smem_raw)[warp];
+
+  int c0 = 0, m = 0, keep = 0;
+  if (valid) {
+    c0 = seq_chunk_ptr[seq_of_chunk(seq_chunk_ptr, num_seqs, i)];
+    m = i - c0;  // admissible candidates c0 .. i-1
+    keep = row_budget(m, budget);
   }
+  if (lane == 0) s_entries[warp] = valid ? keep + 1 : 0;
+  if (threadIdx.x == 0) {
+    // plan entries of every chunk before i0, within one head
+    long long acc = 0;
+    for (int bb = 0; bb < num_seqs; ++bb) {
+      const int cb = seq_chunk_ptr[bb];
+      if (cb >= i0) break;
+      acc += plan_entries(min(seq_chunk_ptr[bb + 1], i0) - cb, budget);
+    }
+    s_base = acc;
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) ws.hist[32 * q + lane] = 0;
+  __syncthreads();
+  if (!valid) return;
+  long long off = s_base + static_cast<long long>(h) * nnz_per_head;
+  for (int w = 0; w < warp; ++w) off += s_entries[w];
+  const int row = h * num_chunks + i;
+  if (lane == 0) {
+    row_ptr[row] = static_cast<int>(off);
+    if (row == num_q_heads * num_chunks - 1) row_ptr[row + 1] = static_cast<int>(off) + keep + 1;
+  }
+  int* out = col + off;
+  if (lane == 0) out[keep] = i;  // the diagonal chunk, last
+  if (keep >= m) {  // every admissible chunk is kept
+    for (int j = lane; j < m; j += 32) out[j] = c0 + j;
+    return;
+  }
+  if (keep == 0) return;
+
+  const float* srow = scores + (static_cast<size_t>(h) * num_chunks + i) * num_chunks + c0;
+  const unsigned lt = (1u << lane) - 1u;
+  int staged = -1;  // keys staged in ws.key / ws.idx, or -1
+  if (m <= kSurvCap) {
+    // short row: stage it whole; first digit histogram fused in
+    for (int j = lane; j < m; j += 32) {
+      const uint32_t k = order_key(__ldcs(srow + j));
+      ws.key[j] = k;
+      ws.idx[j] = static_cast<uint16_t>(j);
+      atomicAdd(&ws.hist[k >> 24], 1);
+    }
+    staged = m;
+  } else if (m <= kFilterMaxCandidates && keep * 8 <= m) {
+    float xv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = 32 * u + lane;
+      xv[u] = j < m ? __ldcs(srow + j) : 0.f;
+    }
+    // threshold from 64 samples at the midpoints of equal strides
+    uint32_t v0 = order_key(__ldg(srow + static_cast<int>(((2LL * lane + 1) * m) / (2 * kSamples))));
+    uint32_t v1 = order_key(__ldg(srow + static_cast<int>(((2LL * (32 + lane) + 1) * m) / (2 * kSamples))));
+    bitonic64_desc(v0, v1, lane);
+    const int r = min(kSamples - 1, static_cast<int>((static_cast<long long>(kSamples) * keep) / m) + kSampleMargin);
+    const float tau = key_float(__shfl_sync(0xffffffffu, r < 32 ? v0 : v1, r & 31));
+    int n = 0;
+    for (int base = 0; base < m; base += 32 * kBatch) {
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = base + 32 * u + lane;
+        const bool sv = j < m && xv[u] >= tau;
+        const unsigned msk = __ballot_sync(0xffffffffu, sv);
+        const int pos = n + __popc(msk & lt);
+        if (sv && pos < kSurvCap) {
+          const uint32_t k = order_key(xv[u]);
+          ws.key[pos] = k;
+          ws.idx[pos] = static_cast<uint16_t>(j);
+          atomicAdd(&ws.hist[k >> 24], 1);
+        }
+        n += __popc(msk);
+      }
+      if (base + 32 * kBatch < m) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = base + 32 * kBatch + 32 * u + lane;
+          xv[u] = j < m ? __ldcs(srow + j) : 0.f;
+        }
+      }
+    }
+    if (n >= keep && n <= kSurvCap) {
+      staged = n;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ws.hist[32 * q + lane] = 0;
+    }
+  }
+  __syncwarp();
+  bool ok;
+  if (staged >= 0) {
+    ok = warp_select(
+        staged, keep, ws.hist, true, [&](int t) { return ws.key[t]; },
+        [&](int t) { return c0 + static_cast<int>(ws.idx[t]); }, out, lane);
+  } else {
+    // select from the row in global memory (read through L2 once per pass)
+    ok = warp_select(
+        m, keep, ws.hist, false, [&](int t) { return order_key(__ldg(srow + t)); },
+        [&](int t) { return c0 + t; }, out, lane);
+  }
+  if (!ok && lane == 0) report(status, kDevCheck);
 }
 
 }  // namespace
 
-size_t topk_select_smem_bytes(int key_capacity) { return static_cast<size_t>(key_capacity) * 4; }
-
 cudaError_t launch_topk_select(const float* scores, int num_chunks, int num_q_heads,
                                const int* seq_chunk_ptr, int num_seqs, BudgetArgs budget,
-                               int* row_ptr, int* col, int nnz_per_head, int key_capacity,
-                               uint32_t* status, cudaStream_t stream) {
+                               int* row_ptr, int* col, int nnz_per_head, uint32_t* status,
+                               cudaStream_t stream) {
   if (num_chunks <= 0) return cudaSuccess;
-  const size_t smem = topk_select_smem_bytes(key_capacity);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid(num_chunks, num_q_heads);
+  constexpr int smem = kSelWarps * static_cast<int>(sizeof(WarpScratch));
+  cudaError_t e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((num_chunks + kSelWarps - 1) / kSelWarps, num_q_heads);
   topk_select_kernel<<<grid, kSelThreads, smem, stream>>>(scores, num_chunks, num_q_heads, seq_chunk_ptr,
                                                              num_seqs, budget, row_ptr, col, nnz_per_head,
-                                                             key_capacity, status);
+                                                             status);
   return cudaGetLastError();
 }
 

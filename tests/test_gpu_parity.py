@@ -106,6 +106,45 @@ def test_topk_select_bit_exact_on_same_scores(name):
                 assert rows[h * n + i] == want, (h, i)
 
 
+def _long_row_scores(n, hq, seed):
+    """Score patterns for rows of hundreds to ~1300 candidates: Gaussian, heavy
+    ties with signed zeros, constant, monotone up and down, rounded Gaussian."""
+    rng = np.random.default_rng(seed)
+    S = np.empty((hq, n, n), dtype=np.float32)
+    S[0] = rng.standard_normal((n, n))
+    S[1] = rng.choice(np.array([-0.0, 0.0, 1.0, 2.0], dtype=np.float32), size=(n, n))
+    S[2] = 0.5
+    S[3] = np.arange(n, dtype=np.float32)[None, :]
+    S[4] = -np.arange(n, dtype=np.float32)[None, :]
+    S[5] = np.round(rng.standard_normal((n, n)), 1)
+    return S
+
+
+@pytest.mark.parametrize("budget", [W.Budget.fraction(1, 20), W.Budget.topk(7), W.Budget.fraction(1, 8),
+                                    W.Budget.topk(1)], ids=["frac5", "top7", "frac12.5", "top1"])
+def test_topk_select_long_rows(budget):
+    """Rows long enough for the sampled-threshold filter, with score patterns
+    that make it succeed (Gaussian, ties inside the survivors, monotone rows)
+    and fail (constant rows overflow the survivor space): every row equals the
+    oracle's selection, bit for bit."""
+    lens = [[1] * 1300, [1] * 600]
+    cu, bounds, sptr = W.make_bounds([1300, 600], lens)
+    hq = 6
+    prob = api.Problem(cu, bounds, sptr, hq, 1, 128, torch.bfloat16, torch.device("cuda"))
+    n = prob.num_chunks
+    S = _long_row_scores(n, hq, 11)
+    plan = api.topk_select(torch.from_numpy(S).cuda(), prob, budget, check=True)
+    rows = gpu_rows(plan, hq * n)
+    for h in range(hq):
+        for bb in range(len(sptr) - 1):
+            c0 = int(sptr[bb])
+            for i in range(c0, int(sptr[bb + 1])):
+                cand = list(range(c0, i))
+                keep = O.row_budget(i - c0, budget.kind, budget.k, budget.num, budget.den)
+                want = sorted(O.select_row([float(S[h, i, j]) for j in cand], cand, keep)) + [i]
+                assert rows[h * n + i] == want, (h, i)
+
+
 @pytest.mark.parametrize("name", CASES)
 def test_plan_and_attention(name):
     inp = _case(name)
