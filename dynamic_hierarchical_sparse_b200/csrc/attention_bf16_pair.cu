@@ -34,8 +34,12 @@
 // O_a at [256 + a*D, 256 + (a+1)*D).  Issue order per key tile t:
 //   PV_0(t), S_0(t+1), PV_1(t), S_1(t+1)
 // so while one warpgroup turns S into P the tensor core works for the other.
-// Online softmax in fp32, exp2 domain, one ex2.approx per element, lazy O
-// rescale (only when a warp's running max grows by more than 2^8).
+// P reaches the tensor core in two halves of 64 keys, each behind its own
+// barrier, so PV_a(t) on the first half runs while the second half is still
+// being exponentiated.
+// Online softmax in fp32, exp2 domain, one ex2.approx per element (the
+// scale-and-shift and the row sums on packed f32x2 FMA / add), lazy O rescale
+// (only when a warp's running max grows by more than 2^8).
 #include "common.cuh"
 #include "exp2_poly.cuh"
 #include "launchers.h"
@@ -54,6 +58,11 @@ constexpr int kPolyPairEvery = 0;
 // Two exponentials per MUFU operation (ex2.approx.f16x2): the arguments are
 // rounded to fp16 (11-bit significand), finer than the bf16 the results feed.
 constexpr bool kExpHalf2 = false;
+// P is handed to the tensor core in two halves of 64 keys: the PV product of
+// the first half runs while the softmax exponentiates the second.
+constexpr bool kSplitP = true;
+// Scale-and-shift of the logits and the row sums on packed f32x2 FMA / add.
+constexpr bool kPackedF32 = true;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -87,8 +96,9 @@ enum {
   kBarSFull = 9,    // + query tile
   kBarPFull = 11,   // + query tile
   kBarOReady = 13,  // + query tile
-  kBarDrain = 15,
-  kNumBars = 16
+  kBarPHalf = 15,   // + query tile: first 64 keys of P written
+  kBarDrain = 17,
+  kNumBars = 18
 };
 
 // Key tiles of one work item: cached runs first, then (if the run list
@@ -167,6 +177,29 @@ __device__ __forceinline__ float2 ex2_pair_f16(float x0, float x1) {
   return r;
 }
 
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// (a.lo * b.lo + c.lo, a.hi * b.hi + c.hi), each rounded once
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -229,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarPFull + s), kBM);
       mbar_init(bar(kBarOReady + s), 1);
+      mbar_init(bar(kBarPHalf + s), kBM);
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -368,17 +402,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int a = 0; ok && a < 2; ++a) {
           const int nta = a == 0 ? nt0 : nt1;
           if (t >= nta) continue;
+          auto issue_pv = [&](int kk0, int kk1) {
+#pragma unroll
+            for (int kk = kk0; kk < kk1; ++kk) {
+              const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, C::kKVSub, 1024);
+              umma_f16_ts(tmem + C::kColO + a * D, tmem + C::kColS + a * 128 + kk * 8, bd, idesc_o,
+                          (t > 0 || kk > 0) ? 1u : 0u);
+            }
+          };
+          if (kSplitP) {
+            if (!mbar_wait(bar(kBarPHalf + a), t & 1, abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(0, kBN / 32);
+          }
           if (!mbar_wait(bar(kBarPFull + a), t & 1, abort_flag, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, C::kKVSub, 1024);
-            umma_f16_ts(tmem + C::kColO + a * D, tmem + C::kColS + a * 128 + kk * 8, bd, idesc_o,
-                        (t > 0 || kk > 0) ? 1u : 0u);
-          }
+          issue_pv(kSplitP ? kBN / 32 : 0, kBN / 16);
           umma_commit(bar(kBarOReady + a));
           if (t + 1 < nta) {
             if (!k_next_ready) {
@@ -475,36 +520,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t ps2[2] = {0ull, 0ull};  // packed (lo, hi) partial sums
+      const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
+      const uint64_t shift2 = f2_pack(-m_use, -m_use);
       uint32_t pk[kBN / 2];
+      // P = exp2(s * scale - m) for columns [cb, cb + 64), packed to bf16 pairs
+      auto exp_cols = [&](int cb) {
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float x0 = fmaf(s[c], scale_log2, -m_use);
-        const float x1 = fmaf(s[c + 1], scale_log2, -m_use);
-        float e0, e1;
-        if (kExpHalf2) {
-          const float2 e = ex2_pair_f16(x0, x1);
-          e0 = e.x;
-          e1 = e.y;
-        } else if (kPolyPairEvery > 0 && (c / 2) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
-          e0 = exp2_fma(x0);
-          e1 = exp2_fma(x1);
-        } else {
-          e0 = ex2_approx(x0);
-          e1 = ex2_approx(x1);
+        for (int c = cb; c < cb + kBN / 2; c += 2) {
+          float x0, x1;
+          if (kPackedF32) {
+            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, shift2), x0, x1);
+          } else {
+            x0 = fmaf(s[c], scale_log2, -m_use);
+            x1 = fmaf(s[c + 1], scale_log2, -m_use);
+          }
+          float e0, e1;
+          if (kExpHalf2) {
+            const float2 e = ex2_pair_f16(x0, x1);
+            e0 = e.x;
+            e1 = e.y;
+          } else if (kPolyPairEvery > 0 && (c / 2) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
+            e0 = exp2_fma(x0);
+            e1 = exp2_fma(x1);
+          } else {
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+          }
+          if (kPackedF32)
+            ps2[(c / 2) & 1] = f2_add(ps2[(c / 2) & 1], f2_pack(e0, e1));
+          else
+            ps[(c / 2) & 3] += e0 + e1;
+          pk[c / 2] = pack_bf16(e0, e1);
         }
-        ps[(c / 2) & 3] += e0 + e1;
-        pk[c / 2] = pack_bf16(e0, e1);
-      }
-      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      // P over the first 64 columns of S (the S values are already in registers)
-      tmem_st32p(tS + 0, pk);
-      tmem_st32p(tS + 32, pk + 32);
-      if (any && t > 0) {
-        // O is rescaled once PV(t-1) has landed
-        if (!mbar_wait(bar(kBarOReady + a), (t - 1) & 1, abort_flag, status)) {
-          ok = false;
-          break;
-        }
+      };
+      // O is rescaled once PV(t-1) has landed, before PV(t) accumulates into it
+      auto rescale_o = [&]() -> bool {
+        if (!mbar_wait(bar(kBarOReady + a), (t - 1) & 1, abort_flag, status)) return false;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -516,6 +568,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(tO + 32 * c, o);
         }
+        return true;
+      };
+      exp_cols(0);
+      // P over the first 64 columns of S (the S values are already in registers)
+      tmem_st32p(tS + 0, pk);
+      if (kSplitP) {
+        if (any && t > 0 && !rescale_o()) {
+          ok = false;
+          break;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPHalf + a));
+      }
+      exp_cols(kBN / 2);
+      tmem_st32p(tS + 32, pk + 32);
+      if (kPackedF32) {
+        float a0, a1, b0, b1;
+        f2_unpack(ps2[0], a0, a1);
+        f2_unpack(ps2[1], b0, b1);
+        l_run = l_run * alpha + ((a0 + a1) + (b0 + b1));
+      } else {
+        l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      }
+      if (!kSplitP && any && t > 0 && !rescale_o()) {
+        ok = false;
+        break;
       }
       tmem_wait_st();
       tc_fence_before();
