@@ -484,9 +484,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[base + 32 + e] = __uint_as_float(rb[e]);
         }
         if (masked) {
+          // only 32-column blocks that reach past the row's last valid column
 #pragma unroll
-          for (int c = base; c < base + kBN / 2; ++c)
-            if (c >= lim) s[c] = -INFINITY;
+          for (int blk = base; blk < base + kBN / 2; blk += 32) {
+            if (lim < blk + 32) {
+#pragma unroll
+              for (int c = blk; c < blk + 32; ++c)
+                if (c >= lim) s[c] = -INFINITY;
+            }
+          }
         }
         // row max as a tree of 3-input maxima (short dependency chains)
 #pragma unroll
