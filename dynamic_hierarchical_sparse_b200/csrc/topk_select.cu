@@ -14,20 +14,22 @@
 // CTA.  Row offsets in the CSR follow from one closed-form offset per CTA
 // (plan_entries) plus the budgets of the CTA's earlier rows.
 //
-// Rows of at most kSurvCap candidates are staged whole in the warp's shared
-// memory as order-preserving 32-bit keys.  Longer rows with a budget of at
-// most 1/8 of the row first try a filter: the warp sorts 64 evenly spaced
-// samples and takes as threshold tau the sample a few ranks below the
-// budget's quantile; one coalesced sweep keeps the keys >= tau ("survivors",
-// in index order).  When at least `keep` keys survive and they fit, the k-th
-// largest key is among them and the exact selection runs on them only;
-// otherwise (an unlucky sample, heavy ties, large budgets) the warp selects
-// from the row in global memory directly, so the result never depends on the
-// sample and no row is too long.  Either way an MSB-first radix select (8-bit
-// digits over a warp-private 256-bin histogram) finds the k-th largest key
-// exactly, stopping early once the threshold bucket is taken whole, and one
-// pass in index order writes the keys above it plus the lowest-indexed keys
-// equal to it.
+// Rows longer than kFilterMin with a budget of at most 1/8 of the row first
+// try a filter: the warp sorts 64 evenly spaced samples and takes as threshold
+// tau the sample a few ranks below the budget's quantile; one coalesced sweep
+// keeps the scores >= tau ("survivors", in index order, with their indices).
+// When at least `keep` scores survive and they fit, the k-th largest score is
+// among them and the exact selection runs on them only.  Otherwise (an unlucky
+// sample, heavy ties, large budgets, short rows) the row is staged whole in the
+// warp's shared memory, or, when it does not fit, selected from global memory
+// directly; so the result never depends on the sample and no row is too long.
+// Every route ends in the same exact selection: an MSB-first radix select over
+// a warp-private 256-bin histogram on order-preserving 32-bit keys.  All keys
+// lie between a known lower bound (tau, or the row minimum) and the row
+// maximum, so they share every bit above the highest bit where the two differ;
+// the radix starts there, takes up to 8 bits per pass and stops once the
+// threshold bucket is taken whole.  One pass in index order then writes the
+// keys above the threshold plus the lowest-indexed keys equal to it.
 #include "common.cuh"
 #include "launchers.h"
 
@@ -37,6 +39,7 @@ namespace {
 constexpr int kSelWarps = 8;  // rows per CTA
 constexpr int kSelThreads = 32 * kSelWarps;
 constexpr int kSurvCap = 896;           // staged keys per warp
+constexpr int kFilterMin = 384;         // rows at most this long are staged whole
 constexpr int kFilterMaxCandidates = 65535;  // survivor indices are 16-bit
 constexpr int kSamples = 64;
 constexpr int kSampleMargin = 5;  // ranks below the budget's sample quantile
@@ -153,28 +156,29 @@ __device__ __forceinline__ void bitonic64_desc(uint32_t& v0, uint32_t& v1, int l
 
 // Exact selection of the `keep` largest of n keys (ties to the lower index),
 // written ascending by index to out[0..keep).  Keys come from get_key(t),
-// their chunk ids from get_col(t), t ascending = index ascending.  hist[] holds
-// the first digit's counts when first_done, else it is zero on entry.
+// their chunk ids from get_col(t), t ascending = index ascending; every key
+// lies in [lo, hi].  The keys then share every bit above the highest bit where
+// lo and hi differ, so the MSB-first radix starts there: each pass takes the
+// (up to) 8 bits below the bits already fixed.  hist[] is zero on entry and is
+// left zero.
 template <typename GetKey, typename GetCol>
-__device__ __forceinline__ bool warp_select(int n, int keep, int* hist, bool first_done, GetKey get_key,
+__device__ __forceinline__ bool warp_select(int n, int keep, uint32_t lo, uint32_t hi, int* hist, GetKey get_key,
                                             GetCol get_col, int* __restrict__ out, int lane) {
-  uint32_t bits = 0, mask = 0;
+  const uint32_t diff = lo ^ hi;
+  int top = diff == 0u ? -1 : 31 - __clz(static_cast<int>(diff));  // highest undecided bit
+  uint32_t mask = top < 0 ? 0xFFFFFFFFu : ~((2u << top) - 1u);      // bits already decided
+  uint32_t bits = lo & mask;
   int remaining = keep;  // still to take among keys matching bits under mask
+  int count = n;         // keys matching bits under mask
 #pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (pass > 0 || !first_done) {
-      if (pass > 0) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) hist[32 * q + lane] = 0;
-        __syncwarp();
-      }
-      for (int t = lane; t < n; t += 32) {
-        const uint32_t k = get_key(t);
-        if ((k & mask) == bits) atomicAdd(&hist[(k >> shift) & 255u], 1);
-      }
-      __syncwarp();
+  while (top >= 0) {
+    const int shift = max(0, top - 7);
+    const uint32_t dmask = (2u << (top - shift)) - 1u;
+    for (int t = lane; t < n; t += 32) {
+      const uint32_t k = get_key(t);
+      if ((k & mask) == bits) atomicAdd(&hist[(k >> shift) & dmask], 1);
     }
+    __syncwarp();
     // lane L owns digits 255-8L down to 248-8L (descending order across lanes)
     int cnt[8];
     int mine = 0;
@@ -183,6 +187,8 @@ __device__ __forceinline__ bool warp_select(int n, int keep, int* hist, bool fir
       cnt[q] = hist[255 - 8 * lane - q];
       mine += cnt[q];
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[255 - 8 * lane - q] = 0;
     int incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -191,7 +197,7 @@ __device__ __forceinline__ bool warp_select(int n, int keep, int* hist, bool fir
     }
     const int excl = incl - mine;
     const bool here = excl < remaining && remaining <= incl;
-    int digit = 0, above = 0, count = 0;
+    int digit = 0, above = 0, cdig = 0;
     if (here) {
       int run = excl;
 #pragma unroll
@@ -199,7 +205,7 @@ __device__ __forceinline__ bool warp_select(int n, int keep, int* hist, bool fir
         if (run + cnt[q] >= remaining) {
           digit = 255 - 8 * lane - q;
           above = run;
-          count = cnt[q];
+          cdig = cnt[q];
           break;
         }
         run += cnt[q];
@@ -208,30 +214,44 @@ __device__ __forceinline__ bool warp_select(int n, int keep, int* hist, bool fir
     const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
     digit = __shfl_sync(0xffffffffu, digit, src);
     above = __shfl_sync(0xffffffffu, above, src);
-    count = __shfl_sync(0xffffffffu, count, src);
+    count = __shfl_sync(0xffffffffu, cdig, src);
     __syncwarp();
     remaining -= above;
     bits |= static_cast<uint32_t>(digit) << shift;
-    mask |= 0xFFu << shift;
+    mask |= dmask << shift;
     if (remaining == count) break;  // the whole bucket is taken: no finer digits needed
+    top = shift - 1;
   }
   // selected: (key & mask) > bits, plus the lowest-indexed `remaining` keys with
-  // (key & mask) == bits (all of them when the bucket was taken whole)
+  // (key & mask) == bits (all of them when the bucket is taken whole)
   const unsigned lt = (1u << lane) - 1u;
-  int written = 0, eq_seen = 0;
-  for (int base = 0; base < n && written < keep; base += 32) {
-    const int t = base + lane;
-    const uint32_t k = t < n ? (get_key(t) & mask) : 0u;
-    const bool gt = t < n && k > bits;
-    const bool eq = t < n && k == bits;
-    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const bool sel = gt || (eq && (eq_seen + __popc(eqm & lt)) < remaining);
-    const unsigned selm = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[written + __popc(selm & lt)] = get_col(t);
-    written += __popc(selm);
-    eq_seen += __popc(eqm);
+  int written = 0;
+  if (remaining == count) {
+    for (int base = 0; base < n && written < keep; base += 32) {
+      const int t = base + lane;
+      const bool sel = t < n && (get_key(t) & mask) >= bits;
+      const unsigned selm = __ballot_sync(0xffffffffu, sel);
+      const int pos = written + __popc(selm & lt);
+      if (sel && pos < keep) out[pos] = get_col(t);
+      written += __popc(selm);
+    }
+  } else {
+    int eq_seen = 0;
+    for (int base = 0; base < n && written < keep; base += 32) {
+      const int t = base + lane;
+      const uint32_t k = t < n ? (get_key(t) & mask) : 0u;
+      const bool gt = t < n && k > bits;
+      const bool eq = t < n && k == bits;
+      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+      const bool sel = gt || (eq && (eq_seen + __popc(eqm & lt)) < remaining);
+      const unsigned selm = __ballot_sync(0xffffffffu, sel);
+      const int pos = written + __popc(selm & lt);
+      if (sel && pos < keep) out[pos] = get_col(t);
+      written += __popc(selm);
+      eq_seen += __popc(eqm);
+    }
   }
-  return written == keep;
+  return written == keep;  // more or fewer would be a defect: reported, never written past the row
 }
 
 // grid: x = group of kSelWarps consecutive chunks, y = query head.
@@ -287,17 +307,8 @@ __global__ void __launch_bounds__(kSelThreads)
 
   const float* srow = scores + (static_cast<size_t>(h) * num_chunks + i) * num_chunks + c0;
   const unsigned lt = (1u << lane) - 1u;
-  int staged = -1;  // keys staged in ws.key / ws.idx, or -1
-  if (m <= kSurvCap) {
-    // short row: stage it whole; first digit histogram fused in
-    for (int j = lane; j < m; j += 32) {
-      const uint32_t k = order_key(__ldcs(srow + j));
-      ws.key[j] = k;
-      ws.idx[j] = static_cast<uint16_t>(j);
-      atomicAdd(&ws.hist[k >> 24], 1);
-    }
-    staged = m;
-  } else if (m <= kFilterMaxCandidates && keep * 8 <= m) {
+  bool ok;
+  if (m > kFilterMin && m <= kFilterMaxCandidates && keep * 8 <= m) {
     float xv[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -309,7 +320,10 @@ __global__ void __launch_bounds__(kSelThreads)
     uint32_t v1 = order_key(__ldg(srow + static_cast<int>(((2LL * (32 + lane) + 1) * m) / (2 * kSamples))));
     bitonic64_desc(v0, v1, lane);
     const int r = min(kSamples - 1, static_cast<int>((static_cast<long long>(kSamples) * keep) / m) + kSampleMargin);
-    const float tau = key_float(__shfl_sync(0xffffffffu, r < 32 ? v0 : v1, r & 31));
+    const uint32_t tau_key = __shfl_sync(0xffffffffu, r < 32 ? v0 : v1, r & 31);
+    const float tau = key_float(tau_key);
+    // sweep: keep the scores >= tau, in index order, as raw bits with their
+    // indices (positions past the space are clamped; such a row falls back)
     int n = 0;
     for (int base = 0; base < m; base += 32 * kBatch) {
 #pragma unroll
@@ -317,12 +331,10 @@ __global__ void __launch_bounds__(kSelThreads)
         const int j = base + 32 * u + lane;
         const bool sv = j < m && xv[u] >= tau;
         const unsigned msk = __ballot_sync(0xffffffffu, sv);
-        const int pos = n + __popc(msk & lt);
-        if (sv && pos < kSurvCap) {
-          const uint32_t k = order_key(xv[u]);
-          ws.key[pos] = k;
+        const int pos = min(n + __popc(msk & lt), kSurvCap - 1);
+        if (sv) {
+          ws.key[pos] = __float_as_uint(xv[u]);
           ws.idx[pos] = static_cast<uint16_t>(j);
-          atomicAdd(&ws.hist[k >> 24], 1);
         }
         n += __popc(msk);
       }
@@ -334,24 +346,62 @@ __global__ void __launch_bounds__(kSelThreads)
         }
       }
     }
+    __syncwarp();
     if (n >= keep && n <= kSurvCap) {
-      staged = n;
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) ws.hist[32 * q + lane] = 0;
+      // every survivor's key is >= tau_key; the row maximum bounds them above
+      uint32_t hi = 0u;
+      for (int t = lane; t < n; t += 32) {
+        const uint32_t k = order_key(__uint_as_float(ws.key[t]));
+        ws.key[t] = k;
+        hi = max(hi, k);
+      }
+      hi = __reduce_max_sync(0xffffffffu, hi);
+      __syncwarp();
+      ok = warp_select(
+          n, keep, tau_key, hi, ws.hist, [&](int t) { return ws.key[t]; },
+          [&](int t) { return c0 + static_cast<int>(ws.idx[t]); }, out, lane);
+      if (!ok && lane == 0) report(status, kDevCheck);
+      return;
     }
   }
-  __syncwarp();
-  bool ok;
-  if (staged >= 0) {
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  if (m <= kSurvCap) {
+    // stage the row whole as order keys, with its key range
+    for (int base = 0; base < m; base += 32 * 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = base + 32 * u + lane;
+        x[u] = j < m ? __ldcs(srow + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = base + 32 * u + lane;
+        if (j < m) {
+          const uint32_t k = order_key(x[u]);
+          ws.key[j] = k;
+          lo = min(lo, k);
+          hi = max(hi, k);
+        }
+      }
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    __syncwarp();
     ok = warp_select(
-        staged, keep, ws.hist, true, [&](int t) { return ws.key[t]; },
-        [&](int t) { return c0 + static_cast<int>(ws.idx[t]); }, out, lane);
+        m, keep, lo, hi, ws.hist, [&](int t) { return ws.key[t]; }, [&](int t) { return c0 + t; }, out, lane);
   } else {
     // select from the row in global memory (read through L2 once per pass)
+    for (int j = lane; j < m; j += 32) {
+      const uint32_t k = order_key(__ldg(srow + j));
+      lo = min(lo, k);
+      hi = max(hi, k);
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
     ok = warp_select(
-        m, keep, ws.hist, false, [&](int t) { return order_key(__ldg(srow + t)); },
-        [&](int t) { return c0 + t; }, out, lane);
+        m, keep, lo, hi, ws.hist, [&](int t) { return order_key(__ldg(srow + t)); }, [&](int t) { return c0 + t; },
+        out, lane);
   }
   if (!ok && lane == 0) report(status, kDevCheck);
 }

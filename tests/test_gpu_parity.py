@@ -145,6 +145,53 @@ def test_topk_select_long_rows(budget):
                 assert rows[h * n + i] == want, (h, i)
 
 
+def _very_long_row_scores(n, hq, seed):
+    """Rows of up to ~3300 candidates (the select micro-benchmark's length):
+    Gaussian, a narrow band where every score shares its sign, exponent and
+    high mantissa bits (the radix must start low), a range over 60 decades,
+    heavy ties with signed zeros, constant, and spikes placed exactly where
+    a sampler with 64 evenly spaced samples looks, so that a sampled threshold
+    keeps too few scores."""
+    rng = np.random.default_rng(seed)
+    S = np.empty((hq, n, n), dtype=np.float32)
+    S[0] = rng.standard_normal((n, n))
+    S[1] = 1000.0 + 1e-3 * rng.standard_normal((n, n))
+    S[2] = rng.standard_normal((n, n)) * 10.0 ** rng.integers(-30, 30, size=(n, n))
+    S[3] = rng.choice(np.array([-0.0, 0.0, 1.0, 2.0], dtype=np.float32), size=(n, n))
+    S[4] = -0.25
+    S[5] = 0.1 * rng.standard_normal((n, n))
+    for i in range(1, n):
+        S[5, i, ((2 * np.arange(64) + 1) * i) // 128] = 10.0
+    return S
+
+
+@pytest.mark.parametrize("budget", [W.Budget.fraction(1, 20), W.Budget.topk(40), W.Budget.fraction(1, 8)],
+                         ids=["frac5", "top40", "frac12.5"])
+def test_topk_select_very_long_rows(budget):
+    """One sequence of 3300 single-token chunks: rows from 0 to 3299
+    candidates through every route (staged, filter, staged after a failed
+    filter, global-memory fallback).  Every 5th row and the last 40 rows of
+    each head are checked against the oracle's selection, bit for bit; every
+    row's length and diagonal are checked."""
+    n_tok = 3300
+    cu, bounds, sptr = W.make_bounds([n_tok], [[1] * n_tok])
+    hq = 6
+    prob = api.Problem(cu, bounds, sptr, hq, 1, 128, torch.bfloat16, torch.device("cuda"))
+    n = prob.num_chunks
+    S = _very_long_row_scores(n, hq, 5)
+    plan = api.topk_select(torch.from_numpy(S).cuda(), prob, budget, check=True)
+    rows = gpu_rows(plan, hq * n)
+    for h in range(hq):
+        for i in range(n):
+            keep = O.row_budget(i, budget.kind, budget.k, budget.num, budget.den)
+            assert len(rows[h * n + i]) == keep + 1 and rows[h * n + i][-1] == i, (h, i)
+            if i % 5 and i < n - 40:
+                continue
+            cand = list(range(i))
+            want = sorted(O.select_row([float(S[h, i, j]) for j in cand], cand, keep)) + [i]
+            assert rows[h * n + i] == want, (h, i)
+
+
 @pytest.mark.parametrize("name", CASES)
 def test_plan_and_attention(name):
     inp = _case(name)
