@@ -22,18 +22,26 @@
 // Warp roles (384 threads = three warpgroups):
 //   warps 0-3   softmax + epilogue of query tile 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of query tile 1
-//   warp 8      TMA producer: both Q tiles once, K/V tiles into 2-stage rings
-//   warp 9      TMEM allocator and the single MMA-issuing thread
-//   warps 10-11 idle
+//   warp 8      TMA producer: both Q tiles once, K tiles into a 2-stage ring,
+//               V tiles into a 3-stage ring; tile t+2 loads once the MMAs
+//               through S(t) are done (one release commit per key tile)
+//   warp 9      TMEM allocator; its lane 0 issues the MMAs of query tile 0
+//   warp 10     lane 0 issues the MMAs of query tile 1
+//   warp 11     idle
 // The launch gives every thread 168 registers (three warps share a
 // sub-partition's 16K); the third warpgroup then hands registers back
 // (setmaxnreg.dec to 56) and the softmax warpgroups take them (224), enough to
 // hold a whole 128-column row of S without spilling.
 // TMEM (512 columns): S_a at [128a, 128a+128); P_a (bf16, two per column) is
 // written over the first 64 columns of S_a and is the A operand of O_a += P_a V;
-// O_a at [256 + a*D, 256 + (a+1)*D).  Issue order per key tile t:
-//   PV_0(t), S_0(t+1), PV_1(t), S_1(t+1)
+// O_a at [256 + a*D, 256 + (a+1)*D).  The tensor pipe takes
+//   PV_0(t), S_0(t+1), PV_1(t), S_1(t+1), PV_0(t+1), ...
 // so while one warpgroup turns S into P the tensor core works for the other.
+// The two issuing threads take turns in that order (a barrier hands the turn
+// over): the pipe queues about one MMA, so a lone issuing thread runs in lock
+// step with it and its own barrier waits and commits between bursts would
+// leave the pipe idle; with two, each passes its waits during the other's
+// turn.  The P barriers take one arrival per softmax warp.
 // P reaches the tensor core in two halves of 64 keys, each behind its own
 // barrier, so PV_a(t) on the first half runs while the second half is still
 // being exponentiated.
@@ -66,7 +74,8 @@ constexpr bool kPackedF32 = true;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kRangeCap = 1024;
+constexpr int kRangeCap = 128;  // runs cached in shared memory; more continue from the plan
+constexpr int kVStages = 3;     // V ring depth (K uses 2)
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
@@ -78,7 +87,7 @@ struct PairCfg {
   static constexpr int kOffQ = 0;  // tile a at kOffQ + a * kQBytes
   static constexpr int kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffRanges = kOffV + 2 * kKVBytes;
+  static constexpr int kOffRanges = kOffV + kVStages * kKVBytes;
   static constexpr int kOffBar = kOffRanges + kRangeCap * 8;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
   static constexpr uint32_t kColS = 0;    // + 128 a
@@ -89,16 +98,16 @@ struct PairCfg {
 
 enum {
   kBarQ = 0,
-  kBarKFull = 1,    // + stage
-  kBarKEmpty = 3,   // + stage
-  kBarVFull = 5,    // + stage
-  kBarVEmpty = 7,   // + stage
-  kBarSFull = 9,    // + query tile
-  kBarPFull = 11,   // + query tile
-  kBarOReady = 13,  // + query tile
-  kBarPHalf = 15,   // + query tile: first 64 keys of P written
-  kBarDrain = 17,
-  kNumBars = 18
+  kBarKFull = 1,    // + K stage (2)
+  kBarVFull = 3,    // + V stage (3)
+  kBarRel = 6,      // + (j & 3): MMAs through S(j) done, so K(j+2) and V(j+2) may load
+  kBarSFull = 10,   // + query tile
+  kBarPFull = 12,   // + query tile
+  kBarOReady = 14,  // + query tile: the last PV done (epilogue)
+  kBarPHalf = 16,   // + query tile: first 64 keys of P written
+  kBarDrain = 18,   // + query tile
+  kBarTurn = 20,    // + query tile: that tile's MMA thread ended a turn
+  kNumBars = 22
 };
 
 // Key tiles of one work item: cached runs first, then (if the run list
@@ -256,15 +265,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarQ), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
-      mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarPFull + s), kBM);
+      mbar_init(bar(kBarPFull + s), 4);  // one arrival per softmax warp
       mbar_init(bar(kBarOReady + s), 1);
-      mbar_init(bar(kBarPHalf + s), kBM);
+      mbar_init(bar(kBarPHalf + s), 4);
     }
-    mbar_init(bar(kBarDrain), 1);
+    for (int s = 0; s < kVStages; ++s) mbar_init(bar(kBarVFull + s), 1);
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kBarRel + s), valid1 ? 2 : 1);  // one commit per MMA thread
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarDrain + s), 1);
+      mbar_init(bar(kBarTurn + s), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -345,38 +356,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       int k0, ke, issued = 0;
       for (int t = 0; w.next(k0, ke); ++t) {
         const int s = t & 1;
-        const uint32_t par = ((t >> 1) & 1) ^ 1;
-        if (!mbar_wait(bar(kBarKEmpty + s), par, abort_flag, status)) break;
+        // K(t) replaces K(t-2), read by S(t-2); V(t) replaces V(t-3), read by
+        // PV(t-3), which was issued before S(t-2): both are free once the
+        // release commit that follows S(t-2) has landed.
+        if (t >= 2) {
+          const int j = t - 2;
+          if (!mbar_wait(bar(kBarRel + (j & 3)), (j >> 2) & 1, abort_flag, status)) break;
+        }
         mbar_arrive_expect_tx(bar(kBarKFull + s), C::kKVBytes);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a)
           tma_load_3d(sbase + C::kOffK + s * C::kKVBytes + a * C::kKVSub, &tm_k, bar(kBarKFull + s), a * 64, g, k0);
-        if (!mbar_wait(bar(kBarVEmpty + s), par, abort_flag, status)) {
-          issued = t + 1;
-          break;
-        }
-        mbar_arrive_expect_tx(bar(kBarVFull + s), C::kKVBytes);
+        const int sv = t % kVStages;
+        mbar_arrive_expect_tx(bar(kBarVFull + sv), C::kKVBytes);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a)
-          tma_load_3d(sbase + C::kOffV + s * C::kKVBytes + a * C::kKVSub, &tm_v, bar(kBarVFull + s), a * 64, g, k0);
+          tma_load_3d(sbase + C::kOffV + sv * C::kKVBytes + a * C::kKVSub, &tm_v, bar(kBarVFull + sv), a * 64, g,
+                      k0);
         issued = t + 1;
       }
       if (*abort_flag) {
         // let copies already in flight land before the CTA exits (bounded)
         volatile int never = 0;
         mbar_wait(bar(kBarQ), 0, &never, nullptr, 10000000ull);
-        for (int t = max(0, issued - 2); t < issued; ++t) {
+        for (int t = max(0, issued - 2); t < issued; ++t)
           mbar_wait(bar(kBarKFull + (t & 1)), (t >> 1) & 1, &never, nullptr, 10000000ull);
-          mbar_wait(bar(kBarVFull + (t & 1)), (t >> 1) & 1, &never, nullptr, 10000000ull);
-        }
+        for (int t = max(0, issued - kVStages); t < issued; ++t)
+          mbar_wait(bar(kBarVFull + t % kVStages), (t / kVStages) & 1, &never, nullptr, 10000000ull);
       }
     }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0 && nt > 0) {
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // One MMA-issuing thread per query tile, taking turns: tile 0's thread
+    // issues PV_0(t) and S_0(t+1), hands over, tile 1's thread issues PV_1(t)
+    // and S_1(t+1), hands back.  The turns keep the two softmax warpgroups
+    // half a period apart (so they do not share the exponential unit); two
+    // threads let each one pass its own waits and commits while the other's
+    // MMAs run, instead of leaving the tensor pipe idle meanwhile.
+    const int a = warp - kMmaWarp;
+    const int nta = a == 0 ? nt0 : nt1;
+    if (lane == 0 && nt > 0 && (a == 0 || valid1)) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 1);
-      auto issue_s = [&](int a, int t) {
-        const uint32_t qbase = sbase + C::kOffQ + a * C::kQBytes;
+      const uint32_t qbase = sbase + C::kOffQ + a * C::kQBytes;
+      auto issue_s = [&](int t) {
         const uint32_t kbase = sbase + C::kOffK + (t & 1) * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -386,22 +408,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(bar(kBarSFull + a));
       };
+      // turn k (0 = the first S, k = t + 1 for key tile t): tile 1's thread
+      // waits for tile 0's turn k, tile 0's thread for tile 1's turn k - 1
+      auto wait_turn = [&](int k) -> bool {
+        if (!valid1) return true;
+        if (a == 1) return mbar_wait_spin(bar(kBarTurn + 0), k & 1, abort_flag, status);
+        if (k == 0) return true;
+        return mbar_wait_spin(bar(kBarTurn + 1), (k - 1) & 1, abort_flag, status);
+      };
+      auto end_turn = [&]() {
+        if (valid1) mbar_arrive(bar(kBarTurn + a));
+      };
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, status);
       if (ok) ok = mbar_wait(bar(kBarKFull + 0), 0, abort_flag, status);
+      if (ok) ok = wait_turn(0);
       if (ok) {
         tc_fence_after();
-        for (int a = 0; a < 2; ++a)
-          if ((a == 0 ? nt0 : nt1) > 0) issue_s(a, 0);
-        umma_commit(bar(kBarKEmpty + 0));
+        if (nta > 0) issue_s(0);
+        umma_commit(bar(kBarRel + 0));  // j = 0: S(0) done
+        end_turn();
       }
       for (int t = 0; ok && t < nt; ++t) {
-        const int s = t & 1;
-        if (!mbar_wait(bar(kBarVFull + s), (t >> 1) & 1, abort_flag, status)) break;
-        const uint32_t vbase = sbase + C::kOffV + s * C::kKVBytes;
-        bool k_next_ready = false;
-        for (int a = 0; ok && a < 2; ++a) {
-          const int nta = a == 0 ? nt0 : nt1;
-          if (t >= nta) continue;
+        const int sv = t % kVStages;
+        if (!mbar_wait_spin(bar(kBarVFull + sv), (t / kVStages) & 1, abort_flag, status)) break;
+        if (t < nta) {
+          const uint32_t vbase = sbase + C::kOffV + sv * C::kKVBytes;
           auto issue_pv = [&](int kk0, int kk1) {
 #pragma unroll
             for (int kk = kk0; kk < kk1; ++kk) {
@@ -410,41 +441,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (t > 0 || kk > 0) ? 1u : 0u);
             }
           };
-          if (kSplitP) {
-            if (!mbar_wait(bar(kBarPHalf + a), t & 1, abort_flag, status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_pv(0, kBN / 32);
-          }
-          if (!mbar_wait(bar(kBarPFull + a), t & 1, abort_flag, status)) {
-            ok = false;
+          if (!mbar_wait_spin(bar(kBarPHalf + a), t & 1, abort_flag, status)) break;
+          if (t + 1 < nta &&
+              !mbar_wait_spin(bar(kBarKFull + ((t + 1) & 1)), ((t + 1) >> 1) & 1, abort_flag, status))
             break;
-          }
+          if (!wait_turn(t + 1)) break;
           tc_fence_after();
-          issue_pv(kSplitP ? kBN / 32 : 0, kBN / 16);
-          umma_commit(bar(kBarOReady + a));
-          if (t + 1 < nta) {
-            if (!k_next_ready) {
-              if (!mbar_wait(bar(kBarKFull + ((t + 1) & 1)), ((t + 1) >> 1) & 1, abort_flag, status)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              k_next_ready = true;
-            }
-            issue_s(a, t + 1);
-          }
+          issue_pv(0, kBN / 32);
+          if (!mbar_wait_spin(bar(kBarPFull + a), t & 1, abort_flag, status)) break;
+          tc_fence_after();
+          issue_pv(kBN / 32, kBN / 16);
+          // only the epilogue waits for O: S(t+1), issued after PV(t), tells
+          // the softmax that PV(t) is done before it rescales O
+          if (t + 1 == nta) umma_commit(bar(kBarOReady + a));
+          if (t + 1 < nta) issue_s(t + 1);
+        } else if (!wait_turn(t + 1)) {
+          break;
         }
-        if (!ok) break;
-        umma_commit(bar(kBarVEmpty + s));
-        if (t + 1 < nt) umma_commit(bar(kBarKEmpty + ((t + 1) & 1)));
+        if (t + 1 < nt) umma_commit(bar(kBarRel + ((t + 1) & 3)));  // j = t + 1: S(t+1) done
+        end_turn();
       }
       // every MMA issued above completes before TMEM is released
-      umma_commit(bar(kBarDrain));
+      umma_commit(bar(kBarDrain + a));
       volatile int never = 0;
-      mbar_wait(bar(kBarDrain), 0, &never, nullptr);
+      mbar_wait(bar(kBarDrain + a), 0, &never, nullptr);
     }
   }
   } else {
@@ -560,10 +580,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c / 2] = pack_bf16(e0, e1);
         }
       };
-      // O is rescaled once PV(t-1) has landed, before PV(t) accumulates into it
+      // O is rescaled before PV(t) accumulates into it; PV(t-1) is done, since
+      // S(t), waited for above, was issued after it
       auto rescale_o = [&]() -> bool {
-        if (!mbar_wait(bar(kBarOReady + a), (t - 1) & 1, abort_flag, status)) return false;
-        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -586,7 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(kBarPHalf + a));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarPHalf + a));
       }
       exp_cols(kBN / 2);
       tmem_st32p(tS + 32, pk + 32);
@@ -604,9 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + a));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarPFull + a));
     }
-    if (ok && nta > 0 && mbar_wait(bar(kBarOReady + a), (nta - 1) & 1, abort_flag, status)) {
+    if (ok && nta > 0 && mbar_wait(bar(kBarOReady + a), 0, abort_flag, status)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const bool valid = t_row < q_end;

@@ -69,6 +69,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (never suspends).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait below, but polls with test_wait instead of try_wait: the
+// thread is never suspended, so it sees a completed phase within a few
+// cycles.  For the one thread whose reaction time is on the critical path.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, uint32_t* status,
+                                               unsigned long long limit_ns = kWaitLimitNs) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u) {
+      if (*abort_flag) return false;
+      if (status != nullptr && (*reinterpret_cast<volatile uint32_t*>(status) & kDevTimeout)) {
+        *abort_flag = 1;
+        return false;
+      }
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        report(status, kDevTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // Waits for the phase with the given parity to complete.  Gives up when the
 // CTA-wide abort flag is set, when another CTA has already recorded a timeout
 // in the global status word, or after limit_ns, setting the flag and the

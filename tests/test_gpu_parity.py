@@ -32,6 +32,12 @@ def _case(name):
         return W.random_problem(4, [1000], 2, 2, 128, "bf16", 50, 300, W.Budget.topk(0))
     if name == "d128_long_runs":
         return W.random_problem(5, [3000], 2, 1, 128, "bf16", 128, 512, W.Budget.fraction(1, 2), "structured")
+    if name == "d128_many_runs":
+        # ~600 chunks of 3-7 tokens, half of each row kept: late rows hold more
+        # than a hundred separate runs of chunks
+        return W.random_problem(8, [3000], 2, 1, 128, "bf16", 3, 7, W.Budget.fraction(1, 2))
+    if name == "d64_many_runs":
+        return W.random_problem(9, [2500], 2, 2, 64, "bf16", 2, 5, W.Budget.fraction(1, 2))
     if name == "tiny_f32":
         return W.generate(W.TINY_1K_F32, 0)
     if name == "f32_d128_ragged":
@@ -40,7 +46,7 @@ def _case(name):
 
 
 CASES = ["ragged_d128_top2", "ragged_d64_frac", "d256_structured_top3", "d128_dense", "d128_diag_only",
-         "d128_long_runs", "tiny_f32", "f32_d128_ragged"]
+         "d128_long_runs", "d128_many_runs", "d64_many_runs", "tiny_f32", "f32_d128_ragged"]
 
 
 @pytest.fixture(scope="module", autouse=True)
