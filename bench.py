@@ -414,6 +414,58 @@ def bench_select_micro(args):
     }), flush=True)
 
 
+def memory_report(spec, seed: int = 0, device=None):
+    """Device memory of one DHSA layer call beyond its inputs and output.
+
+    Returns a dict with the library's size queries (plan workspace, plan
+    arrays, attention workspace), the measured peak of allocations made while
+    planning and attending (torch's allocator statistics, inputs and output
+    allocated beforehand), and, for scale, the bytes of Q/K/V/O and of a dense
+    score matrix [Hq, T, T] in bf16 that attention without tiling would hold.
+    """
+    from dynamic_hierarchical_sparse_b200 import api
+
+    dev = device or torch.device("cuda", 0)
+    inp = W.generate(spec, seed=seed)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    out = torch.empty_like(q)
+    prob = api.Problem.from_inputs(inp, dev)
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    planner = api.Planner(prob, inp.budget, dev)
+    attn = api.Attention(prob, dev)
+    plan = planner(q, k)
+    attn(q, k, v, plan, out)
+    torch.cuda.synchronize(dev)
+    peak_extra = torch.cuda.max_memory_allocated(dev) - base
+    T = int(inp.cu_seqlens[-1])
+    io = (q.numel() + k.numel() + v.numel() + out.numel()) * q.element_size()
+    seq = np.diff(np.asarray(inp.cu_seqlens, dtype=np.int64))
+    rep = {
+        "workload": spec.name, "tokens": T, "num_chunks": inp.num_chunks,
+        "plan_workspace_bytes": prob.plan_workspace_bytes(inp.budget),
+        "plan_bytes": (prob.num_q_heads * prob.num_chunks + 1 + prob.nnz(inp.budget)) * 4,
+        "attention_workspace_bytes": prob.attention_workspace_bytes(),
+        "measured_peak_extra_bytes": int(peak_extra),
+        "qkvo_bytes": int(io),
+        "dense_scores_bf16_bytes": int(spec.num_q_heads * int((seq * seq).sum()) * 2),
+    }
+    rep["extra_over_qkvo"] = rep["measured_peak_extra_bytes"] / io
+    del planner, attn, plan, q, k, v, out
+    torch.cuda.empty_cache()
+    return rep
+
+
+def bench_memory(args):
+    """Peak device memory of plan + attention at each shape (one JSON line each)."""
+    torch.cuda.set_device(0)
+    for spec in (W.GEMMA2_8K, W.LLAMA_32K, W.RAGGED_NEEDLE, W.LLAMA_128K, W.BLOCKSPARSE_128K):
+        rep = memory_report(spec)
+        print(json.dumps(dict(metric="DHSA extra device memory per layer call", unit="bytes",
+                              value=rep["measured_peak_extra_bytes"], higher_is_better=False, **rep)), flush=True)
+
+
 def _budget_str(b):
     if b.kind == W.BUDGET_TOPK:
         return "top-%d + diagonal" % b.k
@@ -461,13 +513,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--memory", action="store_true", help="report device memory per layer call instead")
     ap.add_argument("--micro", default=None, choices=["select"],
                     help="time one kernel alone instead of the full step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3", file=sys.stderr)
         args.warmup = 3
-    if args.micro == "select":
+    if args.memory:
+        bench_memory(args)
+    elif args.micro == "select":
         bench_select_micro(args)
     elif args.impl == "reference":
         bench_reference(args)

@@ -102,7 +102,15 @@ RAGGED_NEEDLE = WorkloadSpec(
     32, 8, 128, "bf16", 64, 512, Budget.topk(8), "normal", needle=True)
 
 WORKLOADS = [TINY_1K_F32, GEMMA2_8K, LLAMA_32K, LLAMA_128K, RAGGED_NEEDLE]
-BY_NAME = {w.name: w for w in WORKLOADS}
+
+# Fixed-length chunks: DHSA with every chunk 512 tokens long is plain
+# block-sparse attention with 512-token blocks (the comparison baseline the
+# pages name), run through the same kernels, on the 128K shape.
+BLOCKSPARSE_128K = WorkloadSpec(
+    "blocksparse512_128k_h32kv8_d128_bf16_frac5", [131072], 32, 8, 128, "bf16", 512,
+    512, Budget.fraction(1, 20), "structured")
+EXTRA_WORKLOADS = [BLOCKSPARSE_128K]
+BY_NAME = {w.name: w for w in WORKLOADS + EXTRA_WORKLOADS}
 
 
 @dataclasses.dataclass

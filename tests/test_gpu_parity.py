@@ -38,6 +38,11 @@ def _case(name):
         return W.random_problem(8, [3000], 2, 1, 128, "bf16", 3, 7, W.Budget.fraction(1, 2))
     if name == "d64_many_runs":
         return W.random_problem(9, [2500], 2, 2, 64, "bf16", 2, 5, W.Budget.fraction(1, 2))
+    if name == "d128_fixed96":
+        # equal chunks of 96 tokens (not a tile multiple) and a shorter last chunk
+        return W.random_problem(10, [2000], 4, 2, 128, "bf16", 96, 96, W.Budget.topk(3), "structured")
+    if name == "d64_fixed256":
+        return W.random_problem(11, [2048, 1024], 2, 1, 64, "bf16", 256, 256, W.Budget.fraction(1, 4))
     if name == "tiny_f32":
         return W.generate(W.TINY_1K_F32, 0)
     if name == "f32_d128_ragged":
@@ -46,7 +51,8 @@ def _case(name):
 
 
 CASES = ["ragged_d128_top2", "ragged_d64_frac", "d256_structured_top3", "d128_dense", "d128_diag_only",
-         "d128_long_runs", "d128_many_runs", "d64_many_runs", "tiny_f32", "f32_d128_ragged"]
+         "d128_long_runs", "d128_many_runs", "d64_many_runs", "d128_fixed96", "d64_fixed256", "tiny_f32",
+         "f32_d128_ragged"]
 
 
 @pytest.fixture(scope="module", autouse=True)
