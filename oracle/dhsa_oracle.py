@@ -41,6 +41,12 @@ ceil(i_local * num / den) chunks (integer arithmetic) capped at i_local; ties go
 to the lower chunk index; plans are per query head (GQA head h reads KV head
 h // (Hq/Hkv)); softmax scale 1/sqrt(d) unless given.
 
+Grouped-query variant (the pages never mention GQA; this is an added mode):
+``per_kv_head=True`` builds one plan row per (KV head g, query chunk i), scored
+by the sum of the chunk scores of g's query heads; every query head of the
+group then attends over that row.  ``group_chunk_scores`` writes the sum out
+head by head.
+
 All arithmetic is numpy float64.  Inputs may be bf16/fp32 torch tensors or
 numpy arrays; they are upcast exactly.
 """
@@ -117,6 +123,20 @@ def chunk_scores(qc: np.ndarray, kc: np.ndarray, seq_chunk_ptr) -> np.ndarray:
     return S
 
 
+def group_chunk_scores(qc: np.ndarray, kc: np.ndarray, seq_chunk_ptr) -> np.ndarray:
+    """Chunk scores of a KV group: S_g[g, i, j] = sum over the query heads h of
+    group g of qc[h, i] . kc[g, j] (same support as ``chunk_scores``)."""
+    S = chunk_scores(qc, kc, seq_chunk_ptr)
+    Hq = qc.shape[0]
+    Hkv = kc.shape[0]
+    group = Hq // Hkv
+    out = np.zeros((Hkv,) + S.shape[1:], dtype=np.float64)
+    for g in range(Hkv):
+        for r in range(group):
+            out[g] += S[g * group + r]
+    return out
+
+
 # ---------------------------------------------------------------- step 3 ---
 def row_budget(i_local: int, kind: int, k: int = 0, num: int = 0, den: int = 1) -> int:
     """How many admissible key chunks a query chunk keeps (diagonal not counted).
@@ -139,12 +159,14 @@ def select_row(scores: Sequence[float], candidates: Sequence[int], keep: int) ->
 
 
 def build_plan(q, k, chunk_bounds, seq_chunk_ptr, budget_kind: int, k_top: int = 0,
-               num: int = 0, den: int = 1):
+               num: int = 0, den: int = 1, per_kv_head: bool = False):
     """The full planning step: representations, scores, per-row selection.
 
     Returns a dict with
       ``row_ptr`` int64 [Hq*n+1] and ``col`` int64 [nnz]: CSR over rows r = h*n+i,
-        each row ascending global chunk ids with the diagonal i last;
+        each row ascending global chunk ids with the diagonal i last (with
+        ``per_kv_head``: [Hkv*n+1] over rows r = g*n+i, scored by
+        ``group_chunk_scores``);
       ``qc``, ``kc``, ``S``: the intermediate fp64 quantities;
       ``kth`` float64 [Hq*n, 2]: the k-th and (k+1)-th best admissible scores of
         the row (NaN where they do not exist), for tie analysis;
@@ -152,8 +174,8 @@ def build_plan(q, k, chunk_bounds, seq_chunk_ptr, budget_kind: int, k_top: int =
     """
     qc = chunk_representations(q, chunk_bounds)
     kc = chunk_representations(k, chunk_bounds)
-    S = chunk_scores(qc, kc, seq_chunk_ptr)
-    Hq, n, _ = qc.shape
+    S = group_chunk_scores(qc, kc, seq_chunk_ptr) if per_kv_head else chunk_scores(qc, kc, seq_chunk_ptr)
+    Hq, n = S.shape[0], S.shape[1]
     ptr = np.asarray(seq_chunk_ptr, dtype=np.int64)
     row_ptr = np.zeros(Hq * n + 1, dtype=np.int64)
     cols: List[int] = []
@@ -197,12 +219,13 @@ def _softmax_rows(logits: np.ndarray) -> np.ndarray:
 
 
 def attention_query_chunk(q, k, v, chunk_bounds, row_ptr, col, h: int, i: int,
-                          scale: Optional[float] = None) -> np.ndarray:
+                          scale: Optional[float] = None, per_kv_head: bool = False) -> np.ndarray:
     """Sparse causal attention of the tokens of query chunk i, head h.
 
-    The kept key chunks' tokens (plan row h*n+i) are concatenated; each query
-    token t attends to the kept tokens s <= t with softmax weights of
-    q_t . k_s * scale and averages v_s.  Returns [L_i, d] float64.
+    The kept key chunks' tokens (plan row h*n+i, or g*n+i for a per-KV-head
+    plan) are concatenated; each query token t attends to the kept tokens
+    s <= t with softmax weights of q_t . k_s * scale and averages v_s.
+    Returns [L_i, d] float64.
     """
     Hq, d = q.shape[1], q.shape[2]
     group = Hq // k.shape[1]
@@ -212,7 +235,8 @@ def attention_query_chunk(q, k, v, chunk_bounds, row_ptr, col, h: int, i: int,
     n = bounds.shape[0] - 1
     rp = np.asarray(row_ptr, dtype=np.int64)
     cl = np.asarray(col, dtype=np.int64)
-    kept = cl[rp[h * n + i]:rp[h * n + i + 1]]
+    r = (g if per_kv_head else h) * n + i
+    kept = cl[rp[r]:rp[r + 1]]
     key_tok = np.concatenate([np.arange(bounds[j], bounds[j + 1]) for j in kept])
     qs = np.arange(bounds[i], bounds[i + 1])
     qq = as_f64(q[int(bounds[i]):int(bounds[i + 1]), h, :])
@@ -224,7 +248,7 @@ def attention_query_chunk(q, k, v, chunk_bounds, row_ptr, col, h: int, i: int,
 
 
 def attention_gather(q, k, v, chunk_bounds, row_ptr, col, scale: Optional[float] = None,
-                     heads: Optional[Iterable[int]] = None) -> np.ndarray:
+                     heads: Optional[Iterable[int]] = None, per_kv_head: bool = False) -> np.ndarray:
     """Sparse causal attention, chunk-gather form, for every query chunk.
 
     Returns O [T, Hq, d] float64 (rows of heads not in ``heads`` stay zero).
@@ -236,12 +260,12 @@ def attention_gather(q, k, v, chunk_bounds, row_ptr, col, scale: Optional[float]
     for h in (range(Hq) if heads is None else heads):
         for i in range(n):
             out[bounds[i]:bounds[i + 1], h, :] = attention_query_chunk(q, k, v, bounds, row_ptr, col, h, i,
-                                                                       scale)
+                                                                       scale, per_kv_head)
     return out
 
 
 def attention_rows(q, k, v, chunk_bounds, row_ptr, col, rows: Sequence[Tuple[int, int]],
-                   scale: Optional[float] = None) -> np.ndarray:
+                   scale: Optional[float] = None, per_kv_head: bool = False) -> np.ndarray:
     """Output of single (token t, head h) rows, one at a time (for large inputs)."""
     d = q.shape[2]
     Hq, Hkv = q.shape[1], k.shape[1]
@@ -255,7 +279,8 @@ def attention_rows(q, k, v, chunk_bounds, row_ptr, col, rows: Sequence[Tuple[int
     for idx, (t, h) in enumerate(rows):
         i = int(np.searchsorted(bounds, t, side="right") - 1)
         g = h // group
-        kept = cl[rp[h * n + i]:rp[h * n + i + 1]]
+        r = (g if per_kv_head else h) * n + i
+        kept = cl[rp[r]:rp[r + 1]]
         key_tok = np.concatenate([np.arange(bounds[j], bounds[j + 1]) for j in kept])
         key_tok = key_tok[key_tok <= t]
         qt = as_f64(q[t, h, :])
@@ -313,17 +338,19 @@ def attention_literal(q, k, v, cu_seqlens, chunk_bounds, seq_chunk_ptr, S: np.nd
     return out, keep, score_tok
 
 
-def kept_pairs(chunk_bounds, row_ptr, col, num_q_heads: int) -> int:
-    """Exact number of (query token, key token, head) pairs the plan keeps."""
+def kept_pairs(chunk_bounds, row_ptr, col, num_q_heads: int, group: int = 1) -> int:
+    """Exact number of (query token, key token, head) pairs the plan keeps.
+
+    ``group`` > 1: a per-KV-head plan whose rows serve ``group`` query heads."""
     bounds = np.asarray(chunk_bounds, dtype=np.int64)
     lens = np.diff(bounds)
     n = lens.shape[0]
     rp = np.asarray(row_ptr, dtype=np.int64)
     cl = np.asarray(col, dtype=np.int64)
     total = 0
-    for r in range(num_q_heads * n):
+    for r in range((num_q_heads // group) * n):
         i = r % n
         Li = int(lens[i])
         for j in cl[rp[r]:rp[r + 1]]:
-            total += Li * (Li + 1) // 2 if j == i else Li * int(lens[j])
+            total += (Li * (Li + 1) // 2 if j == i else Li * int(lens[j])) * group
     return total

@@ -292,6 +292,106 @@ def test_needle_is_selected():
             assert jstar in rows[(g * group) * n + last]
 
 
+# --------------------------------------- grouped-query (per-KV-head) plans
+def _kv_problem(seed, hq=4, hkv=2, d=8):
+    return W.random_problem(seed, [60, 90], hq, hkv, d, "f32", 4, 14, W.Budget.topk(3))
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_kv_plan_equals_head_plan_without_grouping(seed):
+    """With one query head per KV head the group score is the head's score."""
+    inp = _kv_problem(seed, hq=2, hkv=2)
+    b = inp.chunk_bounds
+    p_head = O.build_plan(inp.q, inp.k, b, inp.seq_chunk_ptr, O.TOPK, 3)
+    p_kv = O.build_plan(inp.q, inp.k, b, inp.seq_chunk_ptr, O.TOPK, 3, per_kv_head=True)
+    assert np.array_equal(p_head["row_ptr"], p_kv["row_ptr"]) and np.array_equal(p_head["col"], p_kv["col"])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_kv_plan_with_identical_heads_in_a_group(seed):
+    """When every query head of a group carries the same Q, the group score is
+    the head score times the group size (exact in fp64 for a power of two), so
+    the group's row equals each of its heads' rows."""
+    inp = _kv_problem(seed, hq=4, hkv=2)
+    q = inp.q.clone()
+    q[:, 1] = q[:, 0]
+    q[:, 3] = q[:, 2]
+    b = inp.chunk_bounds
+    n = inp.num_chunks
+    rows_h = O.plan_rows(**{k: v for k, v in O.build_plan(q, inp.k, b, inp.seq_chunk_ptr, O.TOPK, 3).items()
+                            if k in ("row_ptr", "col")})
+    rows_g = O.plan_rows(**{k: v for k, v in O.build_plan(q, inp.k, b, inp.seq_chunk_ptr, O.TOPK, 3,
+                                                          per_kv_head=True).items() if k in ("row_ptr", "col")})
+    assert len(rows_g) == 2 * n
+    for h in range(4):
+        for i in range(n):
+            assert rows_g[(h // 2) * n + i] == rows_h[h * n + i], (h, i)
+
+
+def test_group_scores_are_the_dot_of_summed_query_chunks():
+    """Linearity: the sum over a group's heads of qc[h,i].kc[g,j] equals
+    (sum_h qc[h,i]).kc[g,j]; a wrong head-to-group map breaks it."""
+    inp = _kv_problem(3, hq=6, hkv=2)
+    qc = O.chunk_representations(inp.q, inp.chunk_bounds)
+    kc = O.chunk_representations(inp.k, inp.chunk_bounds)
+    Sg = O.group_chunk_scores(qc, kc, inp.seq_chunk_ptr)
+    summed = qc.reshape(2, 3, qc.shape[1], qc.shape[2]).sum(axis=1)
+    want = np.einsum("gid,gjd->gij", summed, kc)
+    mask = ~np.isnan(Sg)
+    assert mask.sum() > 0 and np.array_equal(mask, ~np.isnan(O.chunk_scores(summed, kc, inp.seq_chunk_ptr)))
+    np.testing.assert_allclose(Sg[mask], want[mask], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("kk", [1, 2, 4])
+def test_kv_plan_matches_brute_force(kk):
+    lens = [3, 1, 4, 2, 5, 1, 3, 2, 4, 2]
+    inp = W.explicit_problem(7, [lens], 4, 2, 8, "f32", W.Budget.topk(kk))
+    p = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, O.TOPK, kk, per_kv_head=True)
+    rows = O.plan_rows(p["row_ptr"], p["col"])
+    qc = O.chunk_representations(inp.q, inp.chunk_bounds)
+    kc = O.chunk_representations(inp.k, inp.chunk_bounds)
+    n = len(lens)
+    for g in range(2):
+        for i in range(n):
+            cands = list(range(i))
+            sc = [float(np.dot(qc[2 * g, i], kc[g, j]) + np.dot(qc[2 * g + 1, i], kc[g, j])) for j in cands]
+            assert rows[g * n + i] == _brute_select(sc, cands, min(kk, i)) + [i]
+
+
+def test_kv_plan_full_budget_equals_dense_causal():
+    """Every query head reads its group's row: with all chunks kept this is
+    dense causal GQA attention (a wrong row lookup reads another group's or a
+    missing row)."""
+    inp = W.random_problem(4, [97, 160], 4, 2, 16, "f32", 5, 40, W.Budget.topk(10 ** 6))
+    q, k, v = (O.as_f64(t) for t in (inp.q, inp.k, inp.v))
+    p = O.build_plan(q, k, inp.chunk_bounds, inp.seq_chunk_ptr, O.TOPK, 10 ** 6, per_kv_head=True)
+    assert p["row_ptr"].shape[0] == 2 * inp.num_chunks + 1
+    got = O.attention_gather(q, k, v, inp.chunk_bounds, p["row_ptr"], p["col"], per_kv_head=True)
+    np.testing.assert_allclose(got, _sdpa_dense(q, k, v, inp.cu_seqlens, 1 / 4.0), rtol=0, atol=1e-12)
+    rows = [(int(t), h) for t in (0, 50, 96, 150, 256) for h in range(4)]
+    np.testing.assert_allclose(O.attention_rows(q, k, v, inp.chunk_bounds, p["row_ptr"], p["col"], rows,
+                                                per_kv_head=True),
+                               np.stack([got[t, h] for t, h in rows]), atol=1e-12)
+    assert O.kept_pairs(inp.chunk_bounds, p["row_ptr"], p["col"], 4, group=2) == 4 * (97 * 98 + 160 * 161) // 2
+
+
+def test_kv_plan_sparse_attention_uses_the_group_row():
+    """With a sparse per-KV-head plan, head h's output equals per-head
+    attention over a plan whose row (h, i) is a copy of row (h // group, i)."""
+    inp = _kv_problem(5, hq=4, hkv=2, d=8)
+    q, k, v = (O.as_f64(t) for t in (inp.q, inp.k, inp.v))
+    b = inp.chunk_bounds
+    n = inp.num_chunks
+    p = O.build_plan(q, k, b, inp.seq_chunk_ptr, O.TOPK, 2, per_kv_head=True)
+    rows = O.plan_rows(p["row_ptr"], p["col"])
+    expanded = [rows[(h // 2) * n + i] for h in range(4) for i in range(n)]
+    rp = np.cumsum([0] + [len(r) for r in expanded])
+    cl = np.asarray([c for r in expanded for c in r])
+    got = O.attention_gather(q, k, v, b, p["row_ptr"], p["col"], per_kv_head=True)
+    want = O.attention_gather(q, k, v, b, rp, cl)
+    np.testing.assert_allclose(got, want, rtol=0, atol=0)
+
+
 # ------------------------------------------------------ planted-mistake check
 def test_planted_mistakes_are_caught(monkeypatch):
     """Each planted slip in the oracle must break at least one pin above."""
@@ -338,6 +438,21 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "select_row", select_low)
     assert not hand_pins_pass()
     monkeypatch.setattr(O, "select_row", real_select)
+
+    # 5) group scores summing the wrong heads (h % Hkv instead of h // group)
+    real_group = O.group_chunk_scores
+
+    def group_wrong(qc, kc, ptr):
+        S = O.chunk_scores(qc, kc, ptr)
+        Hkv = kc.shape[0]
+        out = np.zeros((Hkv,) + S.shape[1:])
+        for h in range(qc.shape[0]):
+            out[h % Hkv] += S[h]
+        return out
+    monkeypatch.setattr(O, "group_chunk_scores", group_wrong)
+    with pytest.raises(AssertionError):
+        test_group_scores_are_the_dot_of_summed_query_chunks()
+    monkeypatch.setattr(O, "group_chunk_scores", real_group)
 
     # 4) softmax without the max shift AND a dropped normaliser
     monkeypatch.setattr(O, "_softmax_rows", lambda lg: np.exp(lg))
