@@ -164,7 +164,7 @@ def whole_job_tokens_per_s(world: int, tokens_per_replica: int, steps: int, max_
     return world * tokens_per_replica * steps / max_elapsed_s
 
 
-def run_cpu_oracle(inp, budget_seconds: float = 20.0):
+def run_cpu_oracle(inp, budget_seconds: float = 20.0, per_kv_head: bool = False):
     """Times the fp64 oracle, as it stands, on a bounded sample of the workload.
 
     Sample: the oracle's full planning step (steps 1-3) on the whole workload,
@@ -176,20 +176,24 @@ def run_cpu_oracle(inp, budget_seconds: float = 20.0):
 
     b = inp.budget
     spec = inp.spec
+    group = spec.num_q_heads // spec.num_kv_heads if per_kv_head else 1
     t0 = time.perf_counter()
-    ref = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, b.kind, b.k, b.num, b.den)
+    ref = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, b.kind, b.k, b.num, b.den,
+                       per_kv_head=per_kv_head)
     t_plan = time.perf_counter() - t0
     n = inp.num_chunks
     lens = np.diff(inp.chunk_bounds.astype(np.int64))
     rp = ref["row_ptr"]
-    total_pairs = kept_pairs(inp.chunk_bounds, rp, ref["col"], n)
+    total_pairs = kept_pairs(inp.chunk_bounds, rp, ref["col"], n) * group
     rng = np.random.default_rng(0)
     order = rng.permutation(spec.num_q_heads * n)
     done_pairs, t_attn, chunks_done = 0, 0.0, 0
-    for r in order:
-        h, i = int(r) // n, int(r) % n
+    for hr in order:
+        h, i = int(hr) // n, int(hr) % n
+        r = (h // group) * n + i
         t1 = time.perf_counter()
-        O.attention_query_chunk(inp.q, inp.k, inp.v, inp.chunk_bounds, rp, ref["col"], h, i)
+        O.attention_query_chunk(inp.q, inp.k, inp.v, inp.chunk_bounds, rp, ref["col"], h, i,
+                                per_kv_head=per_kv_head)
         t_attn += time.perf_counter() - t1
         for j in ref["col"][rp[r]:rp[r + 1]]:
             done_pairs += int(lens[i] * (lens[i] + 1) // 2 if j == i else lens[i] * lens[j])
@@ -226,7 +230,9 @@ def bench_gpu(args):
     dev = torch.device("cuda", local)
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     prob = api.Problem.from_inputs(inp, dev)
-    planner = api.Planner(prob, inp.budget, dev)
+    budget = inp.budget.kv() if args.kv_plan else inp.budget
+    group = spec.num_q_heads // spec.num_kv_heads if args.kv_plan else 1
+    planner = api.Planner(prob, budget, dev)
     attn = api.Attention(prob, dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
@@ -245,7 +251,7 @@ def bench_gpu(args):
     plan = planner(q, k)
     torch.cuda.synchronize()
     pairs = kept_pairs(inp.chunk_bounds, plan.row_ptr.cpu().numpy(), plan.col[:plan.nnz].cpu().numpy(),
-                       inp.num_chunks)
+                       inp.num_chunks) * group
     flops_attn = 4.0 * spec.head_dim * pairs
     reduce_bytes = (q.numel() + k.numel()) * q.element_size()
 
@@ -317,7 +323,7 @@ def bench_gpu(args):
         "config": {
             "workload": spec.name, "tokens": T, "num_seqs": len(spec.seq_lens),
             "q_heads": spec.num_q_heads, "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim,
-            "num_chunks": inp.num_chunks, "budget": _budget_str(inp.budget),
+            "num_chunks": inp.num_chunks, "budget": _budget_str(budget),
             "kept_pairs": pairs, "kept_pairs_frac_of_causal": pairs / (spec.num_q_heads * sum(
                 L * (L + 1) // 2 for L in spec.seq_lens)),
             "parallelism": "replica per GPU" if world > 1 else "single GPU",
@@ -332,7 +338,7 @@ def bench_gpu(args):
             "bound": "tensor", "achieved": achieved_tflops,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved_tflops / peak,
             "peak_kind": "%s bf16 dense, sustained (kernel timed inside a seconds-long loop)" % peaks["source"],
-            "traffic": ATTN_TRAFFIC_BYTES_PER_LAUNCH if spec.name == DEFAULT_WORKLOAD else None,
+            "traffic": ATTN_TRAFFIC_BYTES_PER_LAUNCH if spec.name == DEFAULT_WORKLOAD and not args.kv_plan else None,
             "algorithmic_flops_per_launch": flops_attn,
         },
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -341,7 +347,7 @@ def bench_gpu(args):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = run_cpu_oracle(inp, args.cpu_seconds)
+        result["cpu_baseline"] = run_cpu_oracle(inp, args.cpu_seconds, per_kv_head=args.kv_plan)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -467,9 +473,10 @@ def bench_memory(args):
 
 
 def _budget_str(b):
+    rows = ", one plan row per KV head (group-summed scores)" if getattr(b, "per_kv_head", False) else ""
     if b.kind == W.BUDGET_TOPK:
-        return "top-%d + diagonal" % b.k
-    return "%d/%d of admissible (ceil) + diagonal" % (b.num, b.den)
+        return "top-%d + diagonal%s" % (b.k, rows)
+    return "%d/%d of admissible (ceil) + diagonal%s" % (b.num, b.den, rows)
 
 
 def bench_reference(args):
@@ -484,7 +491,7 @@ def bench_reference(args):
     vals = []
     base = None
     for i in range(args.warmup + args.steps):
-        r = run_cpu_oracle(inp, per_step)
+        r = run_cpu_oracle(inp, per_step, per_kv_head=args.kv_plan)
         if i >= args.warmup:
             vals.append(r["value"])
             base = r
@@ -514,6 +521,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--memory", action="store_true", help="report device memory per layer call instead")
+    ap.add_argument("--kv-plan", action="store_true",
+                    help="grouped-query mode: one plan row per KV head (scored by the group's summed queries)")
     ap.add_argument("--micro", default=None, choices=["select"],
                     help="time one kernel alone instead of the full step")
     args = ap.parse_args()

@@ -31,8 +31,10 @@ EXPORTED = [
     "dhsa_status_string", "dhsa_validate", "dhsa_plan_nnz", "dhsa_chunk_reduce",
     "dhsa_chunk_similarity", "dhsa_topk_select", "dhsa_plan_workspace_size", "dhsa_plan",
     "dhsa_attention_workspace_size", "dhsa_attention", "dhsa_workspace_status",
-    "dhsa_selftest_timeout", "dhsa_plan_noalloc",
+    "dhsa_selftest_timeout", "dhsa_plan_noalloc", "dhsa_attention_kv_plan",
 ]
+
+DHSA_BUDGET_PER_KV_HEAD = 0x100
 
 
 class DhsaError(RuntimeError):
@@ -86,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "dhsa_workspace_status": (ctypes.c_int, [P, P]),
             "dhsa_selftest_timeout": (ctypes.c_int, [P, I32, P]),
             "dhsa_plan_noalloc": (ctypes.c_int, [P, P, PP, _Budget, P, P, I64, P]),
+            "dhsa_attention_kv_plan": (ctypes.c_int, [P, P, P, PP, P, P, I64, ctypes.c_float, P, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -110,7 +113,8 @@ def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
 
 
 def _budget(b: Budget) -> _Budget:
-    return _Budget(int(b.kind), int(b.k), int(b.num), int(b.den))
+    kind = int(b.kind) | (DHSA_BUDGET_PER_KV_HEAD if getattr(b, "per_kv_head", False) else 0)
+    return _Budget(kind, int(b.k), int(b.num), int(b.den))
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -180,9 +184,10 @@ class Problem:
 
 @dataclasses.dataclass
 class Plan:
-    row_ptr: torch.Tensor  # int32 [Hq*n+1] device
+    row_ptr: torch.Tensor  # int32 [Hq*n+1] device ([Hkv*n+1] for a per-KV-head plan)
     col: torch.Tensor      # int32 [nnz] device
     nnz: int
+    per_kv_head: bool = False
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
@@ -221,7 +226,8 @@ def topk_select(scores: torch.Tensor, problem: Problem, budget: Budget, stream=N
     """Step 3 on a given score matrix."""
     nnz = problem.nnz(budget)
     dev = scores.device
-    row_ptr = torch.empty(problem.num_q_heads * problem.num_chunks + 1, dtype=torch.int32, device=dev)
+    heads = problem.num_kv_heads if budget.per_kv_head else problem.num_q_heads
+    row_ptr = torch.empty(heads * problem.num_chunks + 1, dtype=torch.int32, device=dev)
     col = torch.empty(max(nnz, 1), dtype=torch.int32, device=dev)
     ws = _workspace(256, dev)
     st = _stream_ptr(stream)
@@ -229,7 +235,7 @@ def topk_select(scores: torch.Tensor, problem: Problem, budget: Budget, stream=N
                                   nnz, _ptr(ws), ws.numel(), st), "dhsa_topk_select")
     if check:
         _check(lib().dhsa_workspace_status(_ptr(ws), st), "dhsa_topk_select (device)")
-    return Plan(row_ptr, col[:nnz], nnz)
+    return Plan(row_ptr, col[:nnz], nnz, bool(budget.per_kv_head))
 
 
 class Planner:
@@ -240,8 +246,8 @@ class Planner:
         dev = problem.d_bounds.device if device is None else device
         self.nnz = problem.nnz(budget)
         self.ws = _workspace(problem.plan_workspace_bytes(budget), dev)
-        self.row_ptr = torch.empty(problem.num_q_heads * problem.num_chunks + 1, dtype=torch.int32,
-                                   device=dev)
+        heads = problem.num_kv_heads if budget.per_kv_head else problem.num_q_heads
+        self.row_ptr = torch.empty(heads * problem.num_chunks + 1, dtype=torch.int32, device=dev)
         self.col = torch.empty(max(self.nnz, 1), dtype=torch.int32, device=dev)
         self._b = _budget(budget)
 
@@ -249,7 +255,7 @@ class Planner:
         _check(lib().dhsa_plan(_ptr(q), _ptr(k), self.problem.ref(), self._b, _ptr(self.row_ptr),
                                _ptr(self.col), self.nnz, _ptr(self.ws), self.ws.numel(),
                                _stream_ptr(stream)), "dhsa_plan")
-        return Plan(self.row_ptr, self.col[:self.nnz], self.nnz)
+        return Plan(self.row_ptr, self.col[:self.nnz], self.nnz, bool(self.budget.per_kv_head))
 
     def status(self, stream=None) -> int:
         return lib().dhsa_workspace_status(_ptr(self.ws), _stream_ptr(stream))
@@ -264,7 +270,7 @@ def plan(q: torch.Tensor, k: torch.Tensor, problem: Problem, budget: Budget, str
     out = p(q, k, stream)
     if check:
         _check(p.status(stream), "dhsa_plan (device)")
-    return Plan(out.row_ptr.clone(), out.col.clone(), out.nnz)
+    return Plan(out.row_ptr.clone(), out.col.clone(), out.nnz, out.per_kv_head)
 
 
 class Attention:
@@ -277,10 +283,10 @@ class Attention:
 
     def __call__(self, q, k, v, plan: Plan, out: torch.Tensor, scale: Optional[float] = None,
                  stream=None) -> torch.Tensor:
-        _check(lib().dhsa_attention(_ptr(q), _ptr(k), _ptr(v), self.problem.ref(), _ptr(plan.row_ptr),
-                                    _ptr(plan.col), plan.nnz, ctypes.c_float(0.0 if scale is None else scale),
-                                    _ptr(out), _ptr(self.ws), self.ws.numel(), _stream_ptr(stream)),
-               "dhsa_attention")
+        fn = lib().dhsa_attention_kv_plan if plan.per_kv_head else lib().dhsa_attention
+        _check(fn(_ptr(q), _ptr(k), _ptr(v), self.problem.ref(), _ptr(plan.row_ptr), _ptr(plan.col), plan.nnz,
+                  ctypes.c_float(0.0 if scale is None else scale), _ptr(out), _ptr(self.ws), self.ws.numel(),
+                  _stream_ptr(stream)), "dhsa_attention")
         return out
 
     def status(self, stream=None) -> int:

@@ -20,16 +20,26 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int base_kind(const dhsa_budget& b) { return b.kind & 0xFF; }
+bool per_kv_head(const dhsa_budget& b) { return (b.kind & DHSA_BUDGET_PER_KV_HEAD) != 0; }
+
 int64_t budget_of(int i_local, const dhsa_budget& b) {
-  if (b.kind == DHSA_BUDGET_TOPK) return i_local < b.k ? i_local : b.k;
+  if (base_kind(b) == DHSA_BUDGET_TOPK) return i_local < b.k ? i_local : b.k;
   const int64_t want = (static_cast<int64_t>(i_local) * b.num + b.den - 1) / b.den;
   return want < i_local ? want : i_local;
 }
 
 dhsa_status check_budget(const dhsa_budget& b) {
-  if (b.kind == DHSA_BUDGET_TOPK) return b.k >= 0 ? DHSA_OK : DHSA_ERR_INVALID_ARG;
-  if (b.kind == DHSA_BUDGET_FRACTION) return (b.num >= 0 && b.den >= 1) ? DHSA_OK : DHSA_ERR_INVALID_ARG;
+  if ((b.kind & ~(0xFF | DHSA_BUDGET_PER_KV_HEAD)) != 0) return DHSA_ERR_INVALID_ARG;
+  if (base_kind(b) == DHSA_BUDGET_TOPK) return b.k >= 0 ? DHSA_OK : DHSA_ERR_INVALID_ARG;
+  if (base_kind(b) == DHSA_BUDGET_FRACTION) return (b.num >= 0 && b.den >= 1) ? DHSA_OK : DHSA_ERR_INVALID_ARG;
   return DHSA_ERR_INVALID_ARG;
+}
+
+// Plan rows come in blocks of num_chunks, one block per query head, or per KV
+// head for a per-KV-head plan.
+int plan_heads(const dhsa_problem* p, const dhsa_budget& b) {
+  return per_kv_head(b) ? p->num_kv_heads : p->num_q_heads;
 }
 
 dhsa_status check_problem(const dhsa_problem* p) {
@@ -83,30 +93,97 @@ int64_t nnz_per_head(const dhsa_problem* p, const dhsa_budget& b) {
 }
 
 struct PlanLayout {
-  size_t qc, kc, scores, total;
+  size_t qc, kc, qg, scores, total;  // qg: summed query chunks of a per-KV-head plan (else unused)
 };
 
-PlanLayout plan_layout(const dhsa_problem* p) {
+PlanLayout plan_layout(const dhsa_problem* p, const dhsa_budget& b) {
   PlanLayout L;
   const size_t n = static_cast<size_t>(p->num_chunks), d = static_cast<size_t>(p->head_dim);
   L.qc = kStatusBytes;
   L.kc = L.qc + align_up(static_cast<size_t>(p->num_q_heads) * n * d * 4);
-  L.scores = L.kc + align_up(static_cast<size_t>(p->num_kv_heads) * n * d * 4);
-  L.total = L.scores + align_up(static_cast<size_t>(p->num_q_heads) * n * n * 4);
+  L.qg = L.kc + align_up(static_cast<size_t>(p->num_kv_heads) * n * d * 4);
+  L.scores = L.qg + (per_kv_head(b) ? align_up(static_cast<size_t>(p->num_kv_heads) * n * d * 4) : 0);
+  L.total = L.scores + align_up(static_cast<size_t>(plan_heads(p, b)) * n * n * 4);
   return L;
 }
 
 dhsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DHSA_OK : DHSA_ERR_CUDA; }
 
-BudgetArgs to_args(const dhsa_budget& b) { return BudgetArgs{b.kind, b.k, b.num, b.den}; }
+BudgetArgs to_args(const dhsa_budget& b) { return BudgetArgs{base_kind(b), b.k, b.num, b.den}; }
 
-// Selection core shared by dhsa_topk_select and dhsa_plan (after validation).
+// Selection core shared by dhsa_topk_select and the planning steps (after
+// validation): scores [plan_heads, n, n] -> plan rows (plan head, chunk).
 dhsa_status run_select(const float* scores, const dhsa_problem* p, const dhsa_budget& budget, int32_t* row_ptr,
                        int32_t* col, uint32_t* status, cudaStream_t stream) {
   const int64_t per_head = nnz_per_head(p, budget);
-  return cuda_status(launch_topk_select(scores, p->num_chunks, p->num_q_heads, p->seq_chunk_ptr, p->num_seqs,
-                                        to_args(budget), row_ptr, col, static_cast<int>(per_head), status,
-                                        stream));
+  return cuda_status(launch_topk_select(scores, p->num_chunks, plan_heads(p, budget), p->seq_chunk_ptr,
+                                        p->num_seqs, to_args(budget), row_ptr, col, static_cast<int>(per_head),
+                                        status, stream));
+}
+
+// Steps 1-3 into a validated workspace laid out by plan_layout (status word
+// cleared by the caller).
+dhsa_status run_plan(const void* q, const void* k, const dhsa_problem* p, const dhsa_budget& budget,
+                     int32_t* row_ptr, int32_t* col, unsigned char* ws, const PlanLayout& L, cudaStream_t st) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* qc = reinterpret_cast<float*>(ws + L.qc);
+  float* kc = reinterpret_cast<float*>(ws + L.kc);
+  float* scores = reinterpret_cast<float*>(ws + L.scores);
+  cudaError_t e = launch_chunk_reduce(p->dtype, q, p->num_q_heads, qc, k, p->num_kv_heads, kc, p->head_dim,
+                                      p->chunk_bounds, p->num_chunks, st);
+  if (e != cudaSuccess) return DHSA_ERR_CUDA;
+  if (per_kv_head(budget)) {
+    float* qg = reinterpret_cast<float*>(ws + L.qg);
+    e = launch_group_sum(qc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim, qg, st);
+    if (e != cudaSuccess) return DHSA_ERR_CUDA;
+    e = launch_chunk_similarity(qg, kc, p->num_kv_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
+                                p->seq_chunk_ptr, p->num_seqs, scores, st);
+  } else {
+    e = launch_chunk_similarity(qc, kc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
+                                p->seq_chunk_ptr, p->num_seqs, scores, st);
+  }
+  if (e != cudaSuccess) return DHSA_ERR_CUDA;
+  return run_select(scores, p, budget, row_ptr, col, status, st);
+}
+
+// Step 4 after validation; plan_group = query heads per plan row.
+dhsa_status run_attention(const void* q, const void* k, const void* v, const dhsa_problem* p,
+                          const int32_t* row_ptr, const int32_t* col, int64_t nnz, int plan_group, float scale,
+                          void* out, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  if (nnz < static_cast<int64_t>(p->num_q_heads / plan_group) * p->num_chunks)
+    return DHSA_ERR_INVALID_ARG;  // >= diagonal per row
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
+  if (p->total_tokens == 0 || p->num_chunks == 0) return DHSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || row_ptr == nullptr || col == nullptr)
+    return DHSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DHSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(p->head_dim));
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  if (p->dtype == DHSA_F32) {
+    return cuda_status(launch_attention_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                            static_cast<const float*>(v), p->chunk_bounds, p->num_chunks, row_ptr,
+                                            col, p->total_tokens, p->num_q_heads, p->num_kv_heads, p->head_dim,
+                                            plan_group, scale, static_cast<float*>(out), st));
+  }
+  AttnBf16Args a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.bounds = p->chunk_bounds;
+  a.row_ptr = row_ptr;
+  a.col = col;
+  a.num_chunks = p->num_chunks;
+  a.total_tokens = p->total_tokens;
+  a.num_q_heads = p->num_q_heads;
+  a.num_kv_heads = p->num_kv_heads;
+  a.head_dim = p->head_dim;
+  a.max_chunk_len = max_chunk_len(p);
+  a.plan_group = plan_group;
+  a.scale = scale;
+  a.status = status;
+  return cuda_status(launch_attention_bf16(a, st));
 }
 
 __global__ void timeout_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
@@ -188,7 +265,7 @@ dhsa_status dhsa_plan_nnz(const dhsa_problem* p, dhsa_budget budget, int64_t* nn
   dhsa_status s = dhsa_validate(p, &budget);
   if (s != DHSA_OK) return s;
   if (nnz == nullptr) return DHSA_ERR_INVALID_ARG;
-  *nnz = nnz_per_head(p, budget) * p->num_q_heads;
+  *nnz = nnz_per_head(p, budget) * plan_heads(p, budget);
   return DHSA_OK;
 }
 
@@ -220,7 +297,7 @@ dhsa_status dhsa_topk_select(const float* scores, const dhsa_problem* p, dhsa_bu
                              int32_t* col, int64_t nnz, void* workspace, size_t workspace_bytes, void* stream) {
   dhsa_status s = dhsa_validate(p, &budget);
   if (s != DHSA_OK) return s;
-  const int64_t want = nnz_per_head(p, budget) * p->num_q_heads;
+  const int64_t want = nnz_per_head(p, budget) * plan_heads(p, budget);
   if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
   if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
   if (p->num_chunks == 0) return DHSA_OK;
@@ -235,7 +312,7 @@ dhsa_status dhsa_plan_workspace_size(const dhsa_problem* p, dhsa_budget budget, 
   dhsa_status s = dhsa_validate(p, &budget);
   if (s != DHSA_OK) return s;
   if (bytes == nullptr) return DHSA_ERR_INVALID_ARG;
-  *bytes = plan_layout(p).total;
+  *bytes = plan_layout(p, budget).total;
   return DHSA_OK;
 }
 
@@ -243,9 +320,9 @@ dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem* p, dhsa_
                       int32_t* col, int64_t nnz, void* workspace, size_t workspace_bytes, void* stream) {
   dhsa_status s = dhsa_validate(p, &budget);
   if (s != DHSA_OK) return s;
-  const int64_t want = nnz_per_head(p, budget) * p->num_q_heads;
+  const int64_t want = nnz_per_head(p, budget) * plan_heads(p, budget);
   if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
-  const PlanLayout L = plan_layout(p);
+  const PlanLayout L = plan_layout(p, budget);
   if (workspace == nullptr || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return DHSA_ERR_WORKSPACE;
   if (p->num_chunks == 0) return DHSA_OK;
@@ -253,18 +330,8 @@ dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem* p, dhsa_
     return DHSA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  float* qc = reinterpret_cast<float*>(ws + L.qc);
-  float* kc = reinterpret_cast<float*>(ws + L.kc);
-  float* scores = reinterpret_cast<float*>(ws + L.scores);
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
-  cudaError_t e = launch_chunk_reduce(p->dtype, q, p->num_q_heads, qc, k, p->num_kv_heads, kc, p->head_dim,
-                                      p->chunk_bounds, p->num_chunks, st);
-  if (e != cudaSuccess) return DHSA_ERR_CUDA;
-  e = launch_chunk_similarity(qc, kc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
-                              p->seq_chunk_ptr, p->num_seqs, scores, st);
-  if (e != cudaSuccess) return DHSA_ERR_CUDA;
-  return run_select(scores, p, budget, row_ptr, col, status, st);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  return run_plan(q, k, p, budget, row_ptr, col, ws, L, st);
 }
 
 dhsa_status dhsa_attention_workspace_size(const dhsa_problem* p, size_t* bytes) {
@@ -280,39 +347,17 @@ dhsa_status dhsa_attention(const void* q, const void* k, const void* v, const dh
                            void* workspace, size_t workspace_bytes, void* stream) {
   dhsa_status s = check_problem(p);
   if (s != DHSA_OK) return s;
-  if (nnz < static_cast<int64_t>(p->num_q_heads) * p->num_chunks) return DHSA_ERR_INVALID_ARG;  // >= diagonal per row
-  if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
-  if (p->total_tokens == 0 || p->num_chunks == 0) return DHSA_OK;
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || row_ptr == nullptr || col == nullptr)
-    return DHSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DHSA_ERR_INVALID_ARG;
-  if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(p->head_dim));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* status = static_cast<uint32_t*>(workspace);
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
-  if (p->dtype == DHSA_F32) {
-    return cuda_status(launch_attention_f32(static_cast<const float*>(q), static_cast<const float*>(k),
-                                            static_cast<const float*>(v), p->chunk_bounds, p->num_chunks, row_ptr,
-                                            col, p->total_tokens, p->num_q_heads, p->num_kv_heads, p->head_dim,
-                                            scale, static_cast<float*>(out), st));
-  }
-  AttnBf16Args a;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.out = out;
-  a.bounds = p->chunk_bounds;
-  a.row_ptr = row_ptr;
-  a.col = col;
-  a.num_chunks = p->num_chunks;
-  a.total_tokens = p->total_tokens;
-  a.num_q_heads = p->num_q_heads;
-  a.num_kv_heads = p->num_kv_heads;
-  a.head_dim = p->head_dim;
-  a.max_chunk_len = max_chunk_len(p);
-  a.scale = scale;
-  a.status = status;
-  return cuda_status(launch_attention_bf16(a, st));
+  return run_attention(q, k, v, p, row_ptr, col, nnz, 1, scale, out, workspace, workspace_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+dhsa_status dhsa_attention_kv_plan(const void* q, const void* k, const void* v, const dhsa_problem* p,
+                                   const int32_t* row_ptr, const int32_t* col, int64_t nnz, float scale, void* out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  dhsa_status s = check_problem(p);
+  if (s != DHSA_OK) return s;
+  return run_attention(q, k, v, p, row_ptr, col, nnz, p->num_q_heads / p->num_kv_heads, scale, out, workspace,
+                       workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 dhsa_status dhsa_workspace_status(const void* workspace, void* stream) {
@@ -330,9 +375,9 @@ dhsa_status dhsa_plan_noalloc(const void* q, const void* k, const dhsa_problem* 
                               int32_t* row_ptr, int32_t* col, int64_t nnz, void* stream) {
   dhsa_status s = dhsa_validate(p, &budget);
   if (s != DHSA_OK) return s;
-  const int64_t want = nnz_per_head(p, budget) * p->num_q_heads;
+  const int64_t want = nnz_per_head(p, budget) * plan_heads(p, budget);
   if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
-  const PlanLayout L = plan_layout(p);
+  const PlanLayout L = plan_layout(p, budget);
   if (L.total > DHSA_PLAN_NOALLOC_MAX_SCRATCH) return DHSA_ERR_WORKSPACE;  // problem too large for the fixed scratch
   if (p->num_chunks == 0) return DHSA_OK;
   if (q == nullptr || k == nullptr || row_ptr == nullptr || col == nullptr || !aligned16(q) || !aligned16(k))
@@ -342,20 +387,10 @@ dhsa_status dhsa_plan_noalloc(const void* q, const void* k, const dhsa_problem* 
   if (s != DHSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(base);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  float* qc = reinterpret_cast<float*>(ws + L.qc);
-  float* kc = reinterpret_cast<float*>(ws + L.kc);
-  float* scores = reinterpret_cast<float*>(ws + L.scores);
-  // qc, kc and the score triangle are fully rewritten before they are read;
-  // only the status word has to start at zero
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
-  cudaError_t e = launch_chunk_reduce(p->dtype, q, p->num_q_heads, qc, k, p->num_kv_heads, kc, p->head_dim,
-                                      p->chunk_bounds, p->num_chunks, st);
-  if (e != cudaSuccess) return DHSA_ERR_CUDA;
-  e = launch_chunk_similarity(qc, kc, p->num_q_heads, p->num_kv_heads, p->num_chunks, p->head_dim,
-                              p->seq_chunk_ptr, p->num_seqs, scores, st);
-  if (e != cudaSuccess) return DHSA_ERR_CUDA;
-  return run_select(scores, p, budget, row_ptr, col, status, st);
+  // qc, kc, the summed query chunks and the score triangle are fully
+  // rewritten before they are read; only the status word has to start at zero
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  return run_plan(q, k, p, budget, row_ptr, col, ws, L, st);
 }
 
 dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* stream) {

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                           const int* __restrict__ bounds, const int* __restrict__ row_ptr,
                           const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
-                          float scale_log2, uint32_t* status) {
+                          int plan_group, float scale_log2, uint32_t* status) {
   using C = Cfg<D, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (q0 >= c_end) return;  // uniform for the CTA: this chunk has fewer tiles
   const int q_end = min(q0 + kBM, c_end);
   const int g = h / group;
-  const int r = h * num_chunks + ci;
+  const int r = (h / plan_group) * num_chunks + ci;
   const int p0 = row_ptr[r], p1 = row_ptr[r + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -442,7 +442,8 @@ cudaError_t launch_dim(const AttnBf16Args& a, cudaStream_t stream) {
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
                                                   a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
-                                                  a.num_q_heads / a.num_kv_heads, scale_log2, a.status);
+                                                  a.num_q_heads / a.num_kv_heads, a.plan_group, scale_log2,
+                                                  a.status);
   return cudaGetLastError();
 }
 

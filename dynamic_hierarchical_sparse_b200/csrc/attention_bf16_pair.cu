@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                           const int* __restrict__ bounds, const int* __restrict__ row_ptr,
                           const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
-                          float scale_log2, uint32_t* status) {
+                          int plan_group, float scale_log2, uint32_t* status) {
   using C = PairCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q_end1 = valid1 ? min(q0_1 + kBM, c_end) : q0_1;
   const int cap = valid1 ? q_end1 : q_end0;
   const int g = h / group;
-  const int row_id = h * num_chunks + ci;
+  const int row_id = (h / plan_group) * num_chunks + ci;
   const int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -675,7 +675,8 @@ cudaError_t launch_attention_pair_dim(const AttnBf16Args& a, cudaStream_t stream
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
                                                   a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
-                                                  a.num_q_heads / a.num_kv_heads, scale_log2, a.status);
+                                                  a.num_q_heads / a.num_kv_heads, a.plan_group, scale_log2,
+                                                  a.status);
   return cudaGetLastError();
 }
 

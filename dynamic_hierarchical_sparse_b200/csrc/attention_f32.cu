@@ -25,7 +25,8 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
     attention_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                          const float* __restrict__ v, const int* __restrict__ bounds, int num_chunks,
                          const int* __restrict__ row_ptr, const int* __restrict__ col, int total_tokens,
-                         int num_q_heads, int num_kv_heads, float scale, float* __restrict__ out) {
+                         int num_q_heads, int num_kv_heads, int plan_group, float scale,
+                         float* __restrict__ out) {
   constexpr int PER = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kRowsPerCta + warp;
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
 
   const size_t kv_stride = static_cast<size_t>(num_kv_heads) * D;
-  const int r = h * num_chunks + ci;
+  const int r = (h / plan_group) * num_chunks + ci;
   for (int p = row_ptr[r]; p < row_ptr[r + 1]; ++p) {
     const int cj = col[p];
     const int s0 = bounds[cj];
@@ -100,22 +101,25 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
 
 cudaError_t launch_attention_f32(const float* q, const float* k, const float* v, const int* bounds,
                                  int num_chunks, const int* row_ptr, const int* col, int total_tokens,
-                                 int num_q_heads, int num_kv_heads, int head_dim, float scale, float* out,
-                                 cudaStream_t stream) {
+                                 int num_q_heads, int num_kv_heads, int head_dim, int plan_group, float scale,
+                                 float* out, cudaStream_t stream) {
   if (total_tokens <= 0) return cudaSuccess;
   dim3 grid((total_tokens + kRowsPerCta - 1) / kRowsPerCta, num_q_heads);
   switch (head_dim) {
     case 64:
       attention_f32_kernel<64><<<grid, kRowsPerCta * 32, 0, stream>>>(
-          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, scale, out);
+          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, plan_group, scale,
+          out);
       break;
     case 128:
       attention_f32_kernel<128><<<grid, kRowsPerCta * 32, 0, stream>>>(
-          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, scale, out);
+          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, plan_group, scale,
+          out);
       break;
     case 256:
       attention_f32_kernel<256><<<grid, kRowsPerCta * 32, 0, stream>>>(
-          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, scale, out);
+          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, plan_group, scale,
+          out);
       break;
     default:
       return cudaErrorInvalidValue;

@@ -136,4 +136,34 @@ cudaError_t launch_chunk_reduce(int dtype, const void* xa, int heads_a, float* o
                              stream);
 }
 
+namespace {
+
+// Per-KV-head planning scores a KV group by the sum of its query heads' chunk
+// scores, which by linearity is the dot product of the summed query-chunk
+// representations with the KV head's key-chunk representation.
+__global__ void group_sum_kernel(const float* __restrict__ qc, int group, int num_kv_heads, int per_head,
+                                 float* __restrict__ qg) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(num_kv_heads) * per_head) return;
+  const int g = static_cast<int>(idx / per_head);
+  const int e = static_cast<int>(idx - static_cast<int64_t>(g) * per_head);
+  const float* src = qc + static_cast<int64_t>(g) * group * per_head + e;
+  float s = 0.f;
+  for (int r = 0; r < group; ++r) s += src[static_cast<int64_t>(r) * per_head];
+  qg[idx] = s;
+}
+
+}  // namespace
+
+cudaError_t launch_group_sum(const float* qc, int num_q_heads, int num_kv_heads, int num_chunks, int head_dim,
+                             float* qg, cudaStream_t stream) {
+  const int per_head = num_chunks * head_dim;
+  const int64_t total = static_cast<int64_t>(num_kv_heads) * per_head;
+  if (total <= 0) return cudaSuccess;
+  const int threads = 256;
+  group_sum_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, stream>>>(
+      qc, num_q_heads / num_kv_heads, num_kv_heads, per_head, qg);
+  return cudaGetLastError();
+}
+
 }  // namespace dhsa

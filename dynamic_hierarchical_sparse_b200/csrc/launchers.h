@@ -21,6 +21,11 @@ cudaError_t launch_chunk_reduce(int dtype, const void* xa, int heads_a, float* o
                                 int heads_b, float* out_b, int head_dim, const int* bounds,
                                 int num_chunks, cudaStream_t stream);
 
+// Per-KV-head planning: qg[g, c, :] = sum over r < group of qc[g * group + r, c, :]
+// (fp32, fixed order r = 0, 1, ...).
+cudaError_t launch_group_sum(const float* qc, int num_q_heads, int num_kv_heads, int num_chunks, int head_dim,
+                             float* qg, cudaStream_t stream);
+
 // Step 2.
 cudaError_t launch_chunk_similarity(const float* qc, const float* kc, int num_q_heads, int num_kv_heads,
                                     int num_chunks, int head_dim, const int* seq_chunk_ptr,
@@ -32,11 +37,12 @@ cudaError_t launch_topk_select(const float* scores, int num_chunks, int num_q_he
                                int* row_ptr, int* col, int nnz_per_head, uint32_t* status,
                                cudaStream_t stream);
 
-// Step 4, fp32.
+// Step 4, fp32.  plan_group: query heads per plan row (1: a plan row per query
+// head; Hq/Hkv: a plan row per KV head, read by every head of the group).
 cudaError_t launch_attention_f32(const float* q, const float* k, const float* v, const int* bounds,
                                  int num_chunks, const int* row_ptr, const int* col, int total_tokens,
-                                 int num_q_heads, int num_kv_heads, int head_dim, float scale, float* out,
-                                 cudaStream_t stream);
+                                 int num_q_heads, int num_kv_heads, int head_dim, int plan_group, float scale,
+                                 float* out, cudaStream_t stream);
 
 // Step 4, bf16 on tcgen05.  h_bounds is the host mirror of bounds (used to
 // size the grid).
@@ -54,6 +60,7 @@ struct AttnBf16Args {
   int num_kv_heads;
   int head_dim;
   int max_chunk_len;
+  int plan_group;  // query heads per plan row: 1 (per query head) or Hq / Hkv (per KV head)
   float scale;
   uint32_t* status;
 };

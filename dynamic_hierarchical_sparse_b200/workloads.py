@@ -48,12 +48,14 @@ class Budget:
     ``kind == BUDGET_TOPK``: keep ``k`` admissible key chunks.
     ``kind == BUDGET_FRACTION``: keep ``num/den`` of the admissible key chunks
     (rounded up).  The diagonal chunk is kept in addition in both cases.
+    ``per_kv_head``: one plan row per KV head instead of per query head.
     """
 
     kind: int
     k: int = 0
     num: int = 0
     den: int = 1
+    per_kv_head: bool = False  # one plan row per KV head (grouped-query mode)
 
     @staticmethod
     def topk(k: int) -> "Budget":
@@ -62,6 +64,10 @@ class Budget:
     @staticmethod
     def fraction(num: int, den: int) -> "Budget":
         return Budget(BUDGET_FRACTION, num=int(num), den=int(den))
+
+    def kv(self) -> "Budget":
+        """The same budget for a per-KV-head plan."""
+        return dataclasses.replace(self, per_kv_head=True)
 
 
 @dataclasses.dataclass(frozen=True)

@@ -69,6 +69,16 @@ typedef enum { DHSA_BF16 = 0, DHSA_F32 = 1 } dhsa_dtype;
 
 typedef enum { DHSA_BUDGET_TOPK = 0, DHSA_BUDGET_FRACTION = 1 } dhsa_budget_kind;
 
+/* Flag OR-ed into dhsa_budget.kind: a per-KV-head plan.  The pages never
+ * mention grouped-query attention; this is an added mode for GQA models.
+ * Instead of one plan row per (query head h, query chunk i) there is one per
+ * (KV head g, query chunk i), rows r = g * n + i, and its score for key chunk j
+ * is the sum over the query heads h of group g of qc[h, i] . kc[g, j]
+ * (equivalently (sum_h qc[h, i]) . kc[g, j]).  Every query head of the group
+ * then attends over that row: pass the plan to dhsa_attention_kv_plan.  With
+ * Hq == Hkv the two kinds of plan are identical. */
+#define DHSA_BUDGET_PER_KV_HEAD 0x100
+
 /* Key-chunk budget of one query chunk with i_local earlier chunks in its
  * sequence (the diagonal chunk is always kept on top of it):
  *   TOPK:     keep min(k, i_local)
@@ -105,8 +115,9 @@ DHSA_API const char* dhsa_status_string(dhsa_status s);
  * Returns DHSA_OK or the first error found. */
 DHSA_API dhsa_status dhsa_validate(const dhsa_problem* p, const dhsa_budget* budget);
 
-/* Number of plan entries: sum over query heads and chunks of (budget + 1).
- * Host-only, from the host mirrors.  The plan's row count is Hq * n. */
+/* Number of plan entries: sum over plan heads and chunks of (budget + 1).
+ * Host-only, from the host mirrors.  The plan's row count is Hq * n, or
+ * Hkv * n when budget.kind carries DHSA_BUDGET_PER_KV_HEAD. */
 DHSA_API dhsa_status dhsa_plan_nnz(const dhsa_problem* p, dhsa_budget budget, int64_t* nnz);
 
 /* ---- step 1: length-normalised chunk aggregation --------------------------
@@ -133,7 +144,9 @@ DHSA_API dhsa_status dhsa_chunk_similarity(const float* qc, const float* kc,
                                   void* stream);
 
 /* ---- step 3: upsample + select ------------------------------------------
- * For each row r = h * n + i: keep the budget's number of admissible key
+ * For each row r = h * n + i (h < Hq, or h < Hkv with
+ * DHSA_BUDGET_PER_KV_HEAD, where scores are then [Hkv, n, n]): keep the
+ * budget's number of admissible key
  * chunks j < i of i's sequence with the largest scores[h, i, j] (ties to the
  * lower j), plus the diagonal i.  Because every token pair of chunks (i, j)
  * inherits score(i, j), this is the token-level keep set of the pages'
@@ -149,7 +162,9 @@ DHSA_API dhsa_status dhsa_topk_select(const float* scores, const dhsa_problem* p
 
 /* ---- steps 1-3 ------------------------------------------------------------
  * Workspace: dhsa_plan_workspace_size bytes, 256-byte aligned, device.  It
- * holds the status word, qc, kc and the score matrix. */
+ * holds the status word, qc, kc and the score matrix (and, for a per-KV-head
+ * plan, the summed query chunks [Hkv, n, d] fp32; the score matrix is then
+ * [Hkv, n, n]). */
 DHSA_API dhsa_status dhsa_plan_workspace_size(const dhsa_problem* p, dhsa_budget budget,
                                      size_t* bytes);
 DHSA_API dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem* p,
@@ -170,6 +185,14 @@ DHSA_API dhsa_status dhsa_attention(const void* q, const void* k, const void* v,
                            const dhsa_problem* p, const int32_t* row_ptr,
                            const int32_t* col, int64_t nnz, float scale, void* out,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Step 4 over a per-KV-head plan (built with DHSA_BUDGET_PER_KV_HEAD): query
+ * head h reads plan row (h / (Hq/Hkv)) * n + chunk(t).  Arguments, layouts,
+ * workspace and errors as dhsa_attention; nnz is the per-KV-head plan's. */
+DHSA_API dhsa_status dhsa_attention_kv_plan(const void* q, const void* k, const void* v,
+                                           const dhsa_problem* p, const int32_t* row_ptr,
+                                           const int32_t* col, int64_t nnz, float scale, void* out,
+                                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Waits for `stream`, then reads the status word that the kernels of the last
  * call given `workspace` may have set.  Returns DHSA_OK, DHSA_ERR_TIMEOUT or

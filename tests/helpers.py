@@ -74,12 +74,28 @@ def reduce_bound(x, bounds):
     return out
 
 
+def half_ulp_bf16(x):
+    """Half a bf16 ulp at |x| (8 significand bits): the rounding error any
+    bf16 output of value x carries, whatever computed it."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 8)
+
+
+def gate_tolerance(want, dtype):
+    """Per-element gate.  bf16: 2e-2 on the computed attention plus the bf16
+    rounding of the output itself (half an ulp of the reference value; at
+    |O| >= 8 that alone is >= 0.031, above 2e-2).  fp32: 1e-4."""
+    if dtype == torch.bfloat16:
+        return ATOL_BF16 + half_ulp_bf16(want)
+    return np.full(np.shape(want), ATOL_F32)
+
+
 def attention_gate(got, want, dtype):
     """Max-abs error gate; returns (max_err, max|ref|, median|ref|, rel_fro)."""
     g = got.double().cpu().numpy() if hasattr(got, "cpu") else np.asarray(got)
     err = np.abs(g - want)
-    tol = ATOL_BF16 if dtype == torch.bfloat16 else ATOL_F32
+    tol = gate_tolerance(want, dtype)
     stats = (float(err.max()), float(np.abs(want).max()), float(np.median(np.abs(want))),
              float(np.linalg.norm(g - want) / max(np.linalg.norm(want), 1e-30)))
-    assert stats[0] <= tol, ("attention error above gate", stats)
+    assert np.all(err <= tol), ("attention error above gate", stats, float((err - tol).max()))
     return stats

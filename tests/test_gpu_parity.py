@@ -222,6 +222,30 @@ def test_plan_and_attention(name):
     print(name, "max_err=%.3g max|O|=%.3g median|O|=%.3g rel_fro=%.3g" % stats)
 
 
+@pytest.mark.parametrize("name", ["ragged_d128_top2", "ragged_d64_frac", "d256_structured_top3", "d128_many_runs",
+                                  "d128_fixed96", "f32_d128_ragged"])
+def test_per_kv_head_plan_and_attention(name):
+    """Grouped-query mode: one plan row per KV head, scored by the group's
+    summed query chunks, equals the oracle's per-KV-head plan (near-tie rule),
+    and every query head attends over its group's row."""
+    inp = _case(name)
+    q, k, v, prob = to_device(inp)
+    b = inp.budget.kv()
+    plan = api.plan(q, k, prob, b, check=True)
+    assert plan.per_kv_head and plan.row_ptr.numel() == inp.spec.num_kv_heads * inp.num_chunks + 1
+    ref = O.build_plan(inp.q, inp.k, inp.chunk_bounds, inp.seq_chunk_ptr, b.kind, b.k, b.num, b.den,
+                       per_kv_head=True)
+    rows = gpu_rows(plan, inp.spec.num_kv_heads * inp.num_chunks)
+    tolerated = compare_plans(rows, ref, inp, b)
+    assert len(tolerated) <= max(2, len(rows) // 100)
+    out = api.attention(q, k, v, prob, plan, check=True)
+    torch.cuda.synchronize()
+    want = O.attention_gather(inp.q, inp.k, inp.v, inp.chunk_bounds, plan.row_ptr.cpu().numpy(),
+                              plan.col.cpu().numpy(), per_kv_head=True)
+    stats = attention_gate(out, want, inp.q.dtype)
+    print(name, "kv plan: max_err=%.3g max|O|=%.3g" % stats[:2])
+
+
 def test_dense_budget_matches_sdpa():
     inp = _case("d128_dense")
     q, k, v, prob = to_device(inp)

@@ -79,6 +79,23 @@ def test_workspace_sizes():
     assert p.attention_workspace_bytes() >= 256
 
 
+def test_per_kv_head_plan_sizes():
+    """A per-KV-head plan has Hkv*n rows (nnz scales with Hkv, not Hq); its
+    workspace adds the summed query chunks and holds an [Hkv, n, n] score
+    matrix; unknown flag bits are rejected."""
+    inp = W.random_problem(0, [2048, 700], 8, 2, 128, "bf16", 64, 256, W.Budget.topk(4))
+    p = _problem(inp)
+    n = inp.num_chunks
+    for budget in (W.Budget.topk(4), W.Budget.fraction(1, 10)):
+        assert p.nnz(budget.kv()) * 4 == p.nnz(budget)
+    ws = p.plan_workspace_bytes(W.Budget.topk(4).kv())
+    need = 256 + (8 * n * 128 + 2 * n * 128 + 2 * n * 128 + 2 * n * n) * 4
+    assert need <= ws <= need + 5 * 256
+    assert _code(p, W.Budget.topk(4).kv()) == 0
+    bad = W.Budget(W.BUDGET_TOPK | 0x200, k=4)
+    assert _code(p, bad) == 1
+
+
 def _code(problem, budget=None):
     return problem.validate(budget)
 
@@ -226,3 +243,16 @@ def test_closed_form_plan_offsets(budget):
     for L in range(0, 3000):
         assert _plan_entries(L, budget) == running, L
         running += O.row_budget(L, budget.kind, budget.k, budget.num, budget.den) + 1
+
+
+def test_gate_rounding_allowance_is_half_a_bf16_ulp():
+    """The bf16 gate adds the output's own rounding: for any value, rounding
+    to bf16 moves it by at most the allowance, and the allowance is the
+    smallest power of two that always does (a full ulp would be twice it)."""
+    from tests.helpers import half_ulp_bf16
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-3, 3, 20000), [1.0, 4.0, 7.99, 8.0]])
+    r = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.all(np.abs(r - x) <= half_ulp_bf16(x))
+    assert np.abs(r - x).max() > 0.5 * half_ulp_bf16(x[np.argmax(np.abs(r - x))])
+    assert half_ulp_bf16(8.0) == 2.0 ** -5 and half_ulp_bf16(7.99) == 2.0 ** -6
