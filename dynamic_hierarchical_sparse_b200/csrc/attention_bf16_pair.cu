@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                           const int* __restrict__ bounds, const int* __restrict__ row_ptr,
                           const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
-                          int plan_group, float scale_log2, uint32_t* status) {
+                          int plan_group, int head_pair, float scale_log2, uint32_t* status) {
   using C = PairCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -245,17 +245,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   // misc[0] TMEM base, misc[1] abort flag, misc[2] cached runs, misc[3] resume position
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
-  const int pair = blockIdx.x;
-  const int h = blockIdx.y;
+  // Two query tiles per CTA: consecutive 128-row tiles of one head, or, with
+  // head_pair (a plan row per KV group, even group size), the same 128 rows of
+  // two heads 2m and 2m+1 of one group, which then share one key list.
   const int ci = num_chunks - 1 - static_cast<int>(blockIdx.z);  // longest rows first
   const int c_start = bounds[ci], c_end = bounds[ci + 1];
-  const int q0_0 = c_start + pair * 2 * kBM;
+  const int h = head_pair ? 2 * static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);  // tile 0's head
+  const int q0_0 = c_start + static_cast<int>(blockIdx.x) * (head_pair ? 1 : 2) * kBM;
   if (q0_0 >= c_end) return;  // uniform: this chunk has fewer tiles
-  const int q0_1 = q0_0 + kBM;
-  const bool valid1 = q0_1 < c_end;
+  const int q0_1 = head_pair ? q0_0 : q0_0 + kBM;
+  const bool valid1 = head_pair || q0_1 < c_end;
   const int q_end0 = min(q0_0 + kBM, c_end);
   const int q_end1 = valid1 ? min(q0_1 + kBM, c_end) : q0_1;
   const int cap = valid1 ? q_end1 : q_end0;
+  const int h1 = head_pair ? h + 1 : h;  // tile 1's head
   const int g = h / group;
   const int row_id = (h / plan_group) * num_chunks + ci;
   const int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
@@ -349,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (valid1) {
 #pragma unroll
         for (int a = 0; a < D / 64; ++a)
-          tma_load_3d(sbase + C::kOffQ + C::kQBytes + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h, q0_1);
+          tma_load_3d(sbase + C::kOffQ + C::kQBytes + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h1, q0_1);
       }
       TileWalk w;
       w.init(ranges, ncached, col, bounds, resume, p1, cap);
@@ -631,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const bool valid = t_row < q_end;
-      __nv_bfloat16* orow = out + (static_cast<size_t>(t_row) * num_q_heads + h) * D;
+      __nv_bfloat16* orow = out + (static_cast<size_t>(t_row) * num_q_heads + (a == 0 ? h : h1)) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -670,13 +673,15 @@ cudaError_t launch_attention_pair_dim(const AttnBf16Args& a, cudaStream_t stream
   auto kern = attention_pair_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int pairs = (a.max_chunk_len + 2 * kBM - 1) / (2 * kBM);
-  dim3 grid(pairs, a.num_q_heads, a.num_chunks);
+  // a plan row per KV group of even size: pair two heads of the group on the same rows
+  const int head_pair = (a.plan_group >= 2 && a.plan_group % 2 == 0) ? 1 : 0;
+  const int tiles = head_pair ? (a.max_chunk_len + kBM - 1) / kBM : (a.max_chunk_len + 2 * kBM - 1) / (2 * kBM);
+  dim3 grid(tiles, head_pair ? a.num_q_heads / 2 : a.num_q_heads, a.num_chunks);
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
                                                   a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
-                                                  a.num_q_heads / a.num_kv_heads, a.plan_group, scale_log2,
-                                                  a.status);
+                                                  a.num_q_heads / a.num_kv_heads, a.plan_group, head_pair,
+                                                  scale_log2, a.status);
   return cudaGetLastError();
 }
 
