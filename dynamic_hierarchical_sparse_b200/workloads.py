@@ -71,6 +71,21 @@ class Budget:
 
 
 @dataclasses.dataclass(frozen=True)
+class SegmentRule:
+    """Parameters of the online chunking rule.
+
+    Within a sequence, with the current chunk starting at token b, token t
+    starts a new chunk when ``t - b >= max_len``, or when ``t - b >= min_len``
+    and t's adjacent-key similarity (mean over KV heads of cos(k[t-1], k[t]))
+    is below ``threshold``.
+    """
+
+    threshold: float
+    min_len: int
+    max_len: int
+
+
+@dataclasses.dataclass(frozen=True)
 class WorkloadSpec:
     name: str
     seq_lens: Sequence[int]
@@ -268,3 +283,49 @@ def explicit_problem(seed: int, per_seq_chunk_lens: Sequence[Sequence[int]], hq:
     v = torch.randn(T, hkv, d, generator=gen).to(tdtype).contiguous()
     spec = WorkloadSpec("explicit", seq_lens, hq, hkv, d, dtype, 1, 1, budget, values)
     return Inputs(spec, seed, q, k, v, cu, bounds, seq_ptr, budget, None)
+
+
+def planted_segment_keys(seed: int, seq_lens: Sequence[int], hkv: int, d: int, lo: int, hi: int,
+                         dtype: str = "bf16", scale: float = 2.0, noise: float = 0.05):
+    """Keys with planted topic segments, for the online chunking step.
+
+    Segment lengths are drawn U[lo, hi] per sequence (the last one truncated),
+    as for the workloads' chunks.  Every token of a segment has, per KV head,
+    ``scale * u + noise * z``: ``u`` a seeded random unit direction of the
+    segment and head, ``z ~ N(0, 1)`` per token.  Adjacent keys of one segment
+    then have cosine about ``scale^2 / (scale^2 + noise^2 d)`` (0.93 for the
+    defaults at d = 128) and keys of different segments about 0, so a rule
+    with threshold 0.5, min_len = lo and max_len = hi recovers the planted
+    segments.  Returns (k [T, hkv, d], cu_seqlens, chunk_bounds, seq_chunk_ptr)
+    of the planted segments.
+    """
+    rng = np.random.default_rng(seed)
+    per_seq = [chunk_lengths_until(rng, int(L), lo, hi) for L in seq_lens]
+    cu, bounds, seq_ptr = make_bounds(list(seq_lens), per_seq)
+    T = int(cu[-1])
+    n = int(bounds.shape[0] - 1)
+    gen = torch.Generator("cpu").manual_seed(seed)
+    u = torch.randn(n, hkv, d, generator=gen, dtype=torch.float32)
+    u = u / u.norm(dim=-1, keepdim=True)
+    lens = torch.from_numpy(np.diff(bounds).astype(np.int64))
+    k = scale * u.repeat_interleave(lens, dim=0) + noise * torch.randn(T, hkv, d, generator=gen)
+    tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+    return k.to(tdtype).contiguous(), cu, bounds, seq_ptr
+
+
+def drifting_keys(seed: int, T: int, hkv: int, d: int, rho: float = 0.9, dtype: str = "bf16"):
+    """Keys that drift: k[t] = rho * k[t-1] + sqrt(1 - rho^2) * z[t], z ~ N(0, 1).
+
+    Adjacent cosines cluster near ``rho`` with a spread of a few percent, so a
+    threshold near ``rho`` makes many break decisions close to it (the stress
+    case for decisions taken in different precisions)."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    z = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32)
+    k = torch.empty_like(z)
+    if T:
+        k[0] = z[0]
+    c = math.sqrt(1.0 - rho * rho)
+    for t in range(1, T):
+        k[t] = rho * k[t - 1] + c * z[t]
+    tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+    return k.to(tdtype).contiguous()

@@ -47,6 +47,15 @@ by the sum of the chunk scores of g's query heads; every query head of the
 group then attends over that row.  ``group_chunk_scores`` writes the sum out
 head by head.
 
+Online segmentation (step 0; the pages say the sequence is segmented into
+variable-length chunks adaptively and online, but give no rule):
+``segment`` applies this library's stated rule.  Tokens are taken left to
+right within each sequence; with the current chunk starting at token b, token t
+starts a new chunk when t - b >= max_len, or when t - b >= min_len and the
+similarity of t to its predecessor, the mean over KV heads of the cosine of
+k[t-1] and k[t] (``adjacent_key_similarity``), is below the threshold.  A
+zero key has cosine 1 with anything (it never breaks a chunk).
+
 All arithmetic is numpy float64.  Inputs may be bf16/fp32 torch tensors or
 numpy arrays; they are upcast exactly.
 """
@@ -354,3 +363,57 @@ def kept_pairs(chunk_bounds, row_ptr, col, num_q_heads: int, group: int = 1) -> 
         for j in cl[rp[r]:rp[r + 1]]:
             total += (Li * (Li + 1) // 2 if j == i else Li * int(lens[j])) * group
     return total
+
+
+# ------------------------------------------------- step 0 (added mode) ---
+def adjacent_key_similarity(k) -> np.ndarray:
+    """sim[t] = (1/Hkv) sum_g cos(k[t-1, g], k[t, g]) for t >= 1; sim[0] = NaN.
+
+    cos(x, y) = x.y / (|x| |y|), and 1 when either vector is zero.  Sequence
+    edges are not looked at here; ``segment`` never reads sim at a sequence's
+    first token.
+    """
+    K = as_f64(k)
+    T = K.shape[0]
+    sim = np.full(T, np.nan)
+    if T < 2:
+        return sim
+    dot = np.einsum("thd,thd->th", K[:-1], K[1:])
+    norm = np.sqrt(np.einsum("thd,thd->th", K, K))
+    den = norm[:-1] * norm[1:]
+    cos = np.ones_like(dot)
+    nz = den > 0
+    cos[nz] = dot[nz] / den[nz]
+    sim[1:] = cos.mean(axis=1)
+    return sim
+
+
+def segment_sequence(sim: np.ndarray, start: int, end: int, threshold: float, min_len: int,
+                     max_len: int) -> List[int]:
+    """Chunk starts of tokens [start, end) under the greedy online rule."""
+    if end <= start:
+        return []
+    starts = [start]
+    b = start
+    for t in range(start + 1, end):
+        if t - b >= max_len or (t - b >= min_len and sim[t] < threshold):
+            starts.append(t)
+            b = t
+    return starts
+
+
+def segment(k, cu_seqlens, threshold: float, min_len: int, max_len: int):
+    """Online variable-length chunking of every sequence of a packed batch.
+
+    Returns (chunk_bounds int32 [n+1], seq_chunk_ptr int32 [B+1]) in the
+    layout the rest of the path takes.
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    sim = adjacent_key_similarity(k)
+    bounds: List[int] = []
+    ptr = [0]
+    for b in range(cu.shape[0] - 1):
+        bounds += segment_sequence(sim, int(cu[b]), int(cu[b + 1]), threshold, min_len, max_len)
+        ptr.append(len(bounds))
+    bounds.append(int(cu[-1]))
+    return np.asarray(bounds, dtype=np.int32), np.asarray(ptr, dtype=np.int32)
