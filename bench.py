@@ -446,6 +446,77 @@ def bench_select_micro(args):
     }), flush=True)
 
 
+SEGMENT_MICRO = dict(name="segment_micro_128k_kv8_d128_bf16_planted256to1024", tokens=131072, hkv=8, d=128,
+                     lo=256, hi=1024, rule=W.SegmentRule(0.5, 256, 1024))
+
+
+def bench_segment_micro(args):
+    """Online chunking alone on the 128K LLaMA key shape (K [131072, 8, 128]
+    bf16, 268 MB), keys with planted segments U[256, 1024] (the 128K
+    workload's chunk lengths), rule threshold 0.5, min 256, max 1024.  One call
+    is three launches (adjacent-key similarity bits, the walk, compaction).
+    Algorithmic bytes: every key read once plus the two bitmaps written and
+    read (T/8 bytes each way) and the bounds written."""
+    from dynamic_hierarchical_sparse_b200 import api
+    from oracle import dhsa_oracle as O
+
+    cfg = SEGMENT_MICRO
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    k_host, cu, bounds, ptr = W.planted_segment_keys(0, [cfg["tokens"]], cfg["hkv"], cfg["d"], cfg["lo"], cfg["hi"])
+    k = k_host.to(dev)
+    seg = api.Segmenter(cu, cfg["hkv"], cfg["d"], cfg["rule"], dev)
+    b, p, n = seg(k)
+    assert seg.status() == 0
+    n = int(n.item())
+    if not (np.array_equal(b[:n + 1].cpu().numpy(), bounds) and np.array_equal(p.cpu().numpy(), ptr)):
+        raise RuntimeError("segmentation does not recover the planted segments")
+    for _ in range(args.warmup):
+        seg(k)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for _ in range(args.steps):
+        seg(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t = e0.elapsed_time(e1) / 1e3 / args.steps
+    T = cfg["tokens"]
+    key_bytes = T * cfg["hkv"] * cfg["d"] * 2
+    algo = key_bytes + 4 * (T // 8) + 4 * (n + 1) + 4 * 2
+    gbs = algo / t / 1e9
+    peaks = _peaks()
+    res = {
+        "metric": "online chunking HBM GB/s (micro-benchmark)", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_call": t * 1e3, "tokens_per_s": T / t,
+        "higher_is_better": True, "dtype": "bf16 keys, f32 similarity",
+        "data": "synthetic keys with planted segments (seeded)",
+        "config": {"workload": cfg["name"], "tokens": T, "kv_heads": cfg["hkv"], "head_dim": cfg["d"],
+                   "rule": {"threshold": cfg["rule"].threshold, "min_len": cfg["rule"].min_len,
+                            "max_len": cfg["rule"].max_len},
+                   "num_chunks": n, "l2": "no flush: keys %.2f GB > 126 MB L2" % (key_bytes / 1e9)},
+        "roofline": {"kernel": "dhsa_segment (3 launches; adjacent_sim_kernel dominant)", "bound": "hbm",
+                     "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "peak_kind": "%s copy bandwidth" % peaks["source"],
+                     "note": "whole call timed: the walk and compaction count against it"},
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        sample = 16384
+        t0 = time.perf_counter()
+        O.segment(k_host[:sample], [0, sample], cfg["rule"].threshold, cfg["rule"].min_len, cfg["rule"].max_len)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": sample / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                               "sample": "first %d tokens of the same keys" % sample,
+                               "gpu_value_same_unit": T / t}
+    print(json.dumps(res), flush=True)
+
+
 def memory_report(spec, seed: int = 0, device=None):
     """Device memory of one DHSA layer call beyond its inputs and output.
 
@@ -549,7 +620,7 @@ def main():
     ap.add_argument("--memory", action="store_true", help="report device memory per layer call instead")
     ap.add_argument("--kv-plan", action="store_true",
                     help="grouped-query mode: one plan row per KV head (scored by the group's summed queries)")
-    ap.add_argument("--micro", default=None, choices=["select"],
+    ap.add_argument("--micro", default=None, choices=["select", "segment"],
                     help="time one kernel alone instead of the full step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
@@ -559,6 +630,8 @@ def main():
         bench_memory(args)
     elif args.micro == "select":
         bench_select_micro(args)
+    elif args.micro == "segment":
+        bench_segment_micro(args)
     elif args.impl == "reference":
         bench_reference(args)
     else:

@@ -32,6 +32,7 @@ EXPORTED = [
     "dhsa_chunk_similarity", "dhsa_topk_select", "dhsa_plan_workspace_size", "dhsa_plan",
     "dhsa_attention_workspace_size", "dhsa_attention", "dhsa_workspace_status",
     "dhsa_selftest_timeout", "dhsa_plan_noalloc", "dhsa_attention_kv_plan",
+    "dhsa_segment_capacity", "dhsa_segment_workspace_size", "dhsa_segment",
 ]
 
 DHSA_BUDGET_PER_KV_HEAD = 0x100
@@ -57,6 +58,10 @@ class _Problem(ctypes.Structure):
                 ("seq_chunk_ptr", ctypes.c_void_p),
                 ("h_cu_seqlens", ctypes.c_void_p), ("h_chunk_bounds", ctypes.c_void_p),
                 ("h_seq_chunk_ptr", ctypes.c_void_p)]
+
+
+class _SegmentRule(ctypes.Structure):
+    _fields_ = [("threshold", ctypes.c_float), ("min_len", ctypes.c_int32), ("max_len", ctypes.c_int32)]
 
 
 def library_path() -> str:
@@ -89,6 +94,9 @@ def lib() -> ctypes.CDLL:
             "dhsa_selftest_timeout": (ctypes.c_int, [P, I32, P]),
             "dhsa_plan_noalloc": (ctypes.c_int, [P, P, PP, _Budget, P, P, I64, P]),
             "dhsa_attention_kv_plan": (ctypes.c_int, [P, P, P, PP, P, P, I64, ctypes.c_float, P, P, SZ, P]),
+            "dhsa_segment_capacity": (ctypes.c_int, [P, I32, I32, ctypes.POINTER(I64)]),
+            "dhsa_segment_workspace_size": (ctypes.c_int, [I32, ctypes.POINTER(SZ)]),
+            "dhsa_segment": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, _SegmentRule, P, I64, P, P, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -304,6 +312,58 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, problem: Proble
     if check:
         _check(a.status(stream), "dhsa_attention (device)")
     return out
+
+
+class Segmenter:
+    """Owns the buffers of repeated online chunking calls (dhsa_segment) for
+    one batch layout: sequence offsets, KV heads, head dim and rule."""
+
+    def __init__(self, cu_seqlens, num_kv_heads: int, head_dim: int, rule, device=None):
+        self.h_cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        self.num_seqs = int(self.h_cu.shape[0] - 1)
+        self.num_kv_heads, self.head_dim = int(num_kv_heads), int(head_dim)
+        self.rule = rule
+        self._rule = _SegmentRule(float(rule.threshold), int(rule.min_len), int(rule.max_len))
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        L = lib()
+        cap = ctypes.c_int64(0)
+        _check(L.dhsa_segment_capacity(self.h_cu.ctypes.data_as(ctypes.c_void_p), self.num_seqs,
+                                       int(rule.min_len), ctypes.byref(cap)), "dhsa_segment_capacity")
+        self.capacity = int(cap.value)
+        ws = ctypes.c_size_t(0)
+        _check(L.dhsa_segment_workspace_size(int(self.h_cu[-1]), ctypes.byref(ws)), "dhsa_segment_workspace_size")
+        self.ws = _workspace(ws.value, dev)
+        self.d_cu = torch.from_numpy(self.h_cu).to(dev)
+        self.chunk_bounds = torch.empty(self.capacity + 1, dtype=torch.int32, device=dev)
+        self.seq_chunk_ptr = torch.empty(self.num_seqs + 1, dtype=torch.int32, device=dev)
+        self.num_chunks = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def __call__(self, k: torch.Tensor, stream=None):
+        """Asynchronous: returns the device arrays (chunk_bounds holds
+        num_chunks + 1 valid entries)."""
+        _require(k, "k")
+        _check(lib().dhsa_segment(_ptr(k), _dtype_code(k), self.num_kv_heads, self.head_dim, self.num_seqs,
+                                  _ptr(self.d_cu), self.h_cu.ctypes.data_as(ctypes.c_void_p), self._rule,
+                                  _ptr(self.chunk_bounds), self.capacity, _ptr(self.seq_chunk_ptr),
+                                  _ptr(self.num_chunks), _ptr(self.ws), self.ws.numel(), _stream_ptr(stream)),
+               "dhsa_segment")
+        return self.chunk_bounds, self.seq_chunk_ptr, self.num_chunks
+
+    def status(self, stream=None) -> int:
+        return lib().dhsa_workspace_status(_ptr(self.ws), _stream_ptr(stream))
+
+
+def segment(k: torch.Tensor, cu_seqlens, rule, stream=None, check: bool = False):
+    """Online variable-length chunking of the packed batch ``k`` [T, Hkv, d].
+
+    Waits for the result and returns host int32 arrays (chunk_bounds [n+1],
+    seq_chunk_ptr [B+1]), ready for ``Problem``."""
+    seg = Segmenter(cu_seqlens, k.shape[1], k.shape[2], rule, k.device)
+    bounds, ptr, n = seg(k, stream)
+    if check:
+        _check(seg.status(stream), "dhsa_segment (device)")
+    n = int(n.item())
+    return bounds[:n + 1].cpu().numpy(), ptr.cpu().numpy()
 
 
 def selftest_timeout(limit_us: int = 20000, device=None) -> int:

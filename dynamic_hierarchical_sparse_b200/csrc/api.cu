@@ -402,4 +402,60 @@ dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* strea
   return cuda_status(launch_timeout_selftest(status, static_cast<unsigned long long>(limit_us) * 1000ull, st));
 }
 
+dhsa_status dhsa_segment_capacity(const int32_t* h_cu_seqlens, int32_t num_seqs, int32_t min_len,
+                                  int64_t* max_chunks) {
+  if (h_cu_seqlens == nullptr || max_chunks == nullptr || num_seqs < 0 || min_len < 1) return DHSA_ERR_INVALID_ARG;
+  if (h_cu_seqlens[0] != 0) return DHSA_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int b = 0; b < num_seqs; ++b) {
+    const int64_t L = static_cast<int64_t>(h_cu_seqlens[b + 1]) - h_cu_seqlens[b];
+    if (L < 0) return DHSA_ERR_INVALID_ARG;
+    total += (L + min_len - 1) / min_len;
+  }
+  *max_chunks = total;
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_segment_workspace_size(int32_t total_tokens, size_t* bytes) {
+  if (total_tokens < 0 || bytes == nullptr) return DHSA_ERR_INVALID_ARG;
+  const size_t words = (static_cast<size_t>(total_tokens) + 31) / 32;
+  *bytes = kStatusBytes + 2 * align_up(words * sizeof(uint32_t));
+  return DHSA_OK;
+}
+
+dhsa_status dhsa_segment(const void* k, int32_t dtype, int32_t num_kv_heads, int32_t head_dim, int32_t num_seqs,
+                         const int32_t* cu_seqlens, const int32_t* h_cu_seqlens, dhsa_segment_rule rule,
+                         int32_t* chunk_bounds, int64_t max_chunks, int32_t* seq_chunk_ptr, int32_t* num_chunks,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (dtype != DHSA_BF16 && dtype != DHSA_F32) return DHSA_ERR_INVALID_ARG;
+  if (num_kv_heads < 1 || num_seqs < 0) return DHSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) {
+    return head_dim > 0 ? DHSA_ERR_UNSUPPORTED : DHSA_ERR_INVALID_ARG;
+  }
+  if (isnan(rule.threshold) || rule.min_len < 1 || rule.max_len < rule.min_len ||
+      rule.max_len > DHSA_SEGMENT_MAX_LEN)
+    return DHSA_ERR_INVALID_ARG;
+  int64_t cap = 0;
+  dhsa_status s = dhsa_segment_capacity(h_cu_seqlens, num_seqs, rule.min_len, &cap);
+  if (s != DHSA_OK) return s;
+  const int32_t T = h_cu_seqlens[num_seqs];
+  if (max_chunks < cap || max_chunks > INT32_MAX - 1) return DHSA_ERR_INVALID_ARG;
+  if (cu_seqlens == nullptr || chunk_bounds == nullptr || seq_chunk_ptr == nullptr || num_chunks == nullptr)
+    return DHSA_ERR_INVALID_ARG;
+  if (T > 0 && (k == nullptr || !aligned16(k))) return DHSA_ERR_INVALID_ARG;
+  size_t need = 0;
+  dhsa_segment_workspace_size(T, &need);
+  if (workspace == nullptr || workspace_bytes < need) return DHSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  const size_t words = (static_cast<size_t>(T) + 31) / 32;
+  uint32_t* drop = reinterpret_cast<uint32_t*>(ws + kStatusBytes);
+  uint32_t* start_bits = reinterpret_cast<uint32_t*>(ws + kStatusBytes + align_up(words * sizeof(uint32_t)));
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  return cuda_status(launch_segment(k, dtype, T, num_kv_heads, head_dim, cu_seqlens, num_seqs, rule.threshold,
+                                    rule.min_len, rule.max_len, chunk_bounds, max_chunks, seq_chunk_ptr,
+                                    num_chunks, drop, start_bits, status, st));
+}
+
 }  // extern "C"

@@ -70,6 +70,13 @@ cudaError_t launch_attention_pair(const AttnBf16Args& a, cudaStream_t stream);
 // TMA view of a packed THD bf16 tensor (see attention_bf16.cu).
 CUresult encode_qkv_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows);
 
+// Online chunking (three launches: adjacent-key similarity bits, a walk per
+// sequence, compaction).  drop and start_bits: ceil(T / 32) words each.
+cudaError_t launch_segment(const void* k, int dtype, int total_tokens, int num_kv_heads, int head_dim,
+                           const int* cu_seqlens, int num_seqs, float threshold, int min_len, int max_len,
+                           int* chunk_bounds, long long capacity, int* seq_chunk_ptr, int* num_chunks,
+                           uint32_t* drop, uint32_t* start_bits, uint32_t* status, cudaStream_t stream);
+
 // Diagnostic: a kernel whose only wait can never be satisfied, bounded by limit_ns.
 cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);
 

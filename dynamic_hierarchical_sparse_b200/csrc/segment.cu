@@ -1,0 +1,360 @@
+// Online variable-length chunking: proposes the chunk boundaries that the rest
+// of the path takes as input.
+//
+// The pages ("Long-Context Modeling with Dynamic Hierarchical Sparse Attention
+// for On-Device LLMs", Abstract and AI Summary) say that DHSA segments each
+// sequence adaptively and online into variable-length chunks, and give no
+// rule.  The rule built here is a plain left-to-right one, decided as tokens
+// arrive: with the current chunk starting at token b, token t starts a new
+// chunk when t - b >= max_len, or when t - b >= min_len and
+//   sim(t) = (1 / Hkv) * sum_g cos(k[t-1, g], k[t, g])
+// is below the threshold (strict; a zero key has cosine 1).
+//
+// Three launches:
+//  1. adjacent_sim_kernel: sim(t) for every token, four consecutive tokens per
+//     warp (each key row read once per warp, 16-byte vector loads, one squared
+//     norm per row), 32 tokens per CTA; one bit per token ("drop": sim(t) <
+//     threshold) into a bitmap.  HBM-bound: every key row is read once from
+//     DRAM (the row before a warp's first token, read by the neighbouring warp
+//     too, hits in cache).
+//  2. segment_walk_kernel: one CTA per sequence.  The sequence's drop bits are
+//     brought into shared memory by a bulk copy, a window of kWinWords words at
+//     a time, and the CTA tabulates for every word the first drop at or after
+//     it (a suffix minimum).  One thread then walks the rule: from chunk start
+//     b, the next start is the first drop in [b + min_len, b + max_len), else
+//     b + max_len: two shared-memory loads per chunk.  Chunk starts are set in
+//     a second bitmap.
+//  3. segment_compact_kernel: one CTA turns the start bitmap into chunk_bounds
+//     (a block-wide scan of per-thread bit counts), then seq_chunk_ptr by binary
+//     search of each sequence's first token.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace dhsa {
+namespace {
+
+constexpr int kSimWarps = 8;             // warps per CTA; 32 tokens per CTA
+constexpr int kWinWords = 4096;          // walk window: 131072 tokens (max_len <= 65536)
+constexpr int kWalkThreads = 256;
+constexpr int kCompactThreads = 1024;
+
+__device__ __forceinline__ void to_float(const uint4& v, float* f, const __nv_bfloat16*) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(p[i]);
+    f[2 * i] = x.x;
+    f[2 * i + 1] = x.y;
+  }
+}
+
+__device__ __forceinline__ void to_float(const uint4& v, float* f, const float*) {
+  f[0] = __uint_as_float(v.x);
+  f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z);
+  f[3] = __uint_as_float(v.w);
+}
+
+// One warp takes R consecutive tokens tb .. tb+R-1 and reads each of the rows
+// tb-1 .. tb+R-1 once: every row's squared norm is formed once and feeds the
+// two cosines it takes part in.  Lanes form groups of G that cover one head's
+// vectors; P = 32 / G heads per pass over the heads.
+template <typename T, int D>
+__global__ void __launch_bounds__(32 * kSimWarps)
+    adjacent_sim_kernel(const T* __restrict__ k, int total_tokens, int hkv, float threshold,
+                        uint32_t* __restrict__ drop, uint32_t* __restrict__ start_bits) {
+  constexpr int E = 16 / static_cast<int>(sizeof(T));  // elements per 16-byte vector
+  constexpr int V = D / E;                            // vectors per head
+  constexpr int G = V < 32 ? V : 32;                  // lanes per head
+  constexpr int P = 32 / G;                           // heads per pass
+  constexpr int IT = V / G;                           // vectors per lane per head
+  constexpr int F = IT * E;                           // floats per lane per row and pass
+  constexpr int R = 32 / kSimWarps;                   // tokens per warp
+  __shared__ uint32_t s_word;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * 32;
+  const int tb = t0 + warp * R;
+  if (threadIdx.x == 0) s_word = 0u;
+  const uint4* kv = reinterpret_cast<const uint4*>(k);
+  const size_t rowv = static_cast<size_t>(hkv) * V;  // vectors per token row
+  const int sub = lane % G;
+  float acc[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) acc[j] = 0.f;
+  for (int g0 = 0; g0 < hkv; g0 += P) {
+    const int g = g0 + lane / G;
+    const bool on = g < hkv;
+    float x[R + 1][F];
+#pragma unroll
+    for (int r = 0; r <= R; ++r) {
+      const int t = tb - 1 + r;
+      const bool valid = on && t >= 0 && t < total_tokens;
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) u = __ldg(kv + static_cast<size_t>(t) * rowv + g * V + it * G + sub);
+        to_float(u, &x[r][it * E], static_cast<const T*>(nullptr));
+      }
+    }
+    float nrm[R + 1], dot[R];
+#pragma unroll
+    for (int r = 0; r <= R; ++r) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < F; ++e) s = fmaf(x[r][e], x[r][e], s);
+      nrm[r] = s;
+    }
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < F; ++e) s = fmaf(x[j][e], x[j + 1][e], s);
+      dot[j] = s;
+    }
+#pragma unroll
+    for (int o = G / 2; o >= 1; o >>= 1) {
+#pragma unroll
+      for (int r = 0; r <= R; ++r) nrm[r] += __shfl_xor_sync(0xffffffffu, nrm[r], o);
+#pragma unroll
+      for (int j = 0; j < R; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], o);
+    }
+    if (sub == 0 && on) {
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        acc[j] += (nrm[j] > 0.f && nrm[j + 1] > 0.f) ? dot[j] * rsqrtf(nrm[j]) * rsqrtf(nrm[j + 1]) : 1.f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+  }
+  __syncthreads();  // s_word initialised
+  if (lane == 0) {
+    uint32_t bits = 0u;
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int t = tb + j;
+      if (t >= 1 && t < total_tokens && acc[j] / static_cast<float>(hkv) < threshold) bits |= 1u << (warp * R + j);
+    }
+    if (bits) atomicOr(&s_word, bits);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    drop[blockIdx.x] = s_word;
+    start_bits[blockIdx.x] = 0u;
+  }
+}
+
+__global__ void __launch_bounds__(kWalkThreads)
+    segment_walk_kernel(const uint32_t* __restrict__ drop, const int* __restrict__ cu_seqlens, int min_len,
+                        int max_len, uint32_t* __restrict__ start_bits, uint32_t* status) {
+  __shared__ __align__(128) uint32_t win[kWinWords];
+  __shared__ int nd[kWinWords + 1];  // nd[i]: first drop at or after word wb + i (in the window), else kNone
+  __shared__ int s_carry[kWalkThreads / 32];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_abort, s_b, s_done;
+  constexpr int kNone = 0x7fffffff;
+  const int seq = blockIdx.x;
+  const int s0 = cu_seqlens[seq], s1 = cu_seqlens[seq + 1];
+  if (s1 <= s0) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int last_word = (s1 - 1) >> 5;
+  const uint32_t mbar = smem_u32(&bar);
+  if (tid == 0) {
+    s_abort = 0;
+    mbar_init(mbar, 1);
+    fence_mbar_init();
+    atomicOr(start_bits + (s0 >> 5), 1u << (s0 & 31));
+  }
+  __syncthreads();
+  int b = s0;
+  int wb = -1;  // first word held in the window (a multiple of 4: 16-byte copies)
+  uint32_t phase = 0;
+  while (true) {
+    const int lo = b + min_len;
+    if (lo >= s1) break;
+    const int hi = min(b + max_len, s1);
+    if (wb < 0 || ((hi - 1) >> 5) >= wb + kWinWords) {
+      // [lo, hi) spans at most (max_len + 29) / 32 + 1 words and wb is at most
+      // 3 words below lo's word, so the new window holds it
+      wb = (lo >> 5) & ~3;
+      const int n = min(kWinWords, last_word + 1 - wb);
+      const uint32_t bytes = static_cast<uint32_t>((n + 3) & ~3) * 4u;  // inside the 256-byte-aligned bitmap
+      __syncthreads();  // every thread is done with the old window
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(mbar, bytes);
+        bulk_load_1d(smem_u32(win), drop + wb, bytes, mbar);
+      }
+      const bool ok = mbar_wait(mbar, phase, &s_abort, status);
+      phase ^= 1u;
+      if (__syncthreads_or(!ok)) return;  // recorded in the status word
+      // nd = suffix minimum of each word's first drop: within each thread's
+      // run of words, then across threads (a suffix-min scan), then patched
+      constexpr int kPer = kWinWords / kWalkThreads;
+      const int i0 = tid * kPer, i1 = min(n, i0 + kPer);
+      int run = kNone;
+      for (int i = i1 - 1; i >= i0; --i) {
+        const uint32_t m = win[i];
+        if (m != 0u) run = ((wb + i) << 5) + __ffs(m) - 1;
+        nd[i] = run;
+      }
+      int suf = run;  // suffix minimum over threads tid .. (inclusive) in this warp
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf = min(suf, v);
+      }
+      if (lane == 0) s_carry[warp] = suf;
+      __syncthreads();
+      int carry = __shfl_down_sync(0xffffffffu, suf, 1);
+      if (lane == 31) carry = kNone;
+      for (int w = warp + 1; w < kWalkThreads / 32; ++w) carry = min(carry, s_carry[w]);
+      for (int i = i0; i < i1; ++i)
+        if (nd[i] == kNone) nd[i] = carry;
+      if (tid == 0) nd[n] = kNone;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      // the walk: two shared-memory loads per chunk
+      int cb = b, done = 0;
+      while (true) {
+        const int clo = cb + min_len;
+        if (clo >= s1) { done = 1; break; }
+        const int chi = min(cb + max_len, s1);
+        const int wl = clo >> 5;
+        if (((chi - 1) >> 5) >= wb + kWinWords) break;  // the window must move first
+        const uint32_t m = win[wl - wb] & (0xffffffffu << (clo & 31));
+        const int f = m != 0u ? (wl << 5) + __ffs(m) - 1 : nd[wl - wb + 1];
+        int next;
+        if (f < chi) {
+          next = f;
+        } else if (cb + max_len < s1) {
+          next = cb + max_len;
+        } else {
+          done = 1;
+          break;
+        }
+        atomicOr(start_bits + (next >> 5), 1u << (next & 31));
+        cb = next;
+      }
+      s_b = cb;
+      s_done = done;
+    }
+    __syncthreads();
+    b = s_b;
+    const int fin = s_done;
+    __syncthreads();  // s_b / s_done are rewritten by the next round
+    if (fin) break;
+  }
+}
+
+__global__ void __launch_bounds__(kCompactThreads)
+    segment_compact_kernel(const uint32_t* __restrict__ start_bits, int total_tokens,
+                           const int* __restrict__ cu_seqlens, int num_seqs, int* __restrict__ chunk_bounds,
+                           long long capacity, int* __restrict__ seq_chunk_ptr, int* __restrict__ num_chunks,
+                           uint32_t* status) {
+  __shared__ int s_warp[kCompactThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = (total_tokens + 31) >> 5;
+  const int per = (nw + kCompactThreads - 1) / kCompactThreads;
+  const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(start_bits[w]);
+  // block-wide exclusive scan of cnt
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int x = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += v;
+    }
+    s_warp[lane] = x;  // inclusive over warps
+  }
+  __syncthreads();
+  const int total = s_warp[kCompactThreads / 32 - 1];
+  long long pos = incl - cnt + (warp > 0 ? s_warp[warp - 1] : 0);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = start_bits[w];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < capacity) chunk_bounds[pos] = (w << 5) + b;
+      ++pos;
+    }
+  }
+  if (tid == 0) {
+    if (total > capacity) report(status, kDevCheck);
+    chunk_bounds[min(static_cast<long long>(total), capacity)] = total_tokens;
+    *num_chunks = total;
+  }
+  __syncthreads();  // chunk_bounds visible to the whole block
+  const int n = static_cast<int>(min(static_cast<long long>(total), capacity));
+  for (int s = tid; s <= num_seqs; s += kCompactThreads) {
+    if (s == num_seqs) {
+      seq_chunk_ptr[s] = n;
+      continue;
+    }
+    const int x = cu_seqlens[s];
+    int lo = 0, hi = n;  // first chunk whose start is >= x
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (chunk_bounds[mid] < x) lo = mid + 1;
+      else hi = mid;
+    }
+    seq_chunk_ptr[s] = lo;
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_sim(const void* k, int total_tokens, int hkv, float threshold, uint32_t* drop,
+                       uint32_t* start_bits, cudaStream_t stream) {
+  const int words = (total_tokens + 31) / 32;
+  adjacent_sim_kernel<T, D><<<words, 32 * kSimWarps, 0, stream>>>(static_cast<const T*>(k), total_tokens, hkv,
+                                                                  threshold, drop, start_bits);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_segment(const void* k, int dtype, int total_tokens, int num_kv_heads, int head_dim,
+                           const int* cu_seqlens, int num_seqs, float threshold, int min_len, int max_len,
+                           int* chunk_bounds, long long capacity, int* seq_chunk_ptr, int* num_chunks,
+                           uint32_t* drop, uint32_t* start_bits, uint32_t* status, cudaStream_t stream) {
+  cudaError_t e = cudaSuccess;
+  if (total_tokens > 0) {
+    if (dtype == 0) {
+      if (head_dim == 64) e = launch_sim<__nv_bfloat16, 64>(k, total_tokens, num_kv_heads, threshold, drop, start_bits, stream);
+      else if (head_dim == 128) e = launch_sim<__nv_bfloat16, 128>(k, total_tokens, num_kv_heads, threshold, drop, start_bits, stream);
+      else e = launch_sim<__nv_bfloat16, 256>(k, total_tokens, num_kv_heads, threshold, drop, start_bits, stream);
+    } else {
+      if (head_dim == 64) e = launch_sim<float, 64>(k, total_tokens, num_kv_heads, threshold, drop, start_bits, stream);
+      else if (head_dim == 128) e = launch_sim<float, 128>(k, total_tokens, num_kv_heads, threshold, drop, start_bits, stream);
+      else e = launch_sim<float, 256>(k, total_tokens, num_kv_heads, threshold, drop, start_bits, stream);
+    }
+    if (e != cudaSuccess) return e;
+    if (num_seqs > 0) {
+      segment_walk_kernel<<<num_seqs, kWalkThreads, 0, stream>>>(drop, cu_seqlens, min_len, max_len, start_bits,
+                                                                 status);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+  }
+  segment_compact_kernel<<<1, kCompactThreads, 0, stream>>>(start_bits, total_tokens, cu_seqlens, num_seqs,
+                                                           chunk_bounds, capacity, seq_chunk_ptr, num_chunks,
+                                                           status);
+  return cudaGetLastError();
+}
+
+}  // namespace dhsa

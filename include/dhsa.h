@@ -18,7 +18,8 @@
  *   4. sparse attention   dhsa_attention         (causal softmax attention over
  *      the kept token pairs only)
  *
- * dhsa_plan runs steps 1-3 back to back.
+ * dhsa_plan runs steps 1-3 back to back.  dhsa_segment (optional) proposes the
+ * chunk boundaries online from the keys, under a rule stated with it.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -205,6 +206,52 @@ DHSA_API dhsa_status dhsa_workspace_status(const void* workspace, void* stream);
  * of `workspace` (>= 256 bytes) and returns.  Exercises the timeout path of
  * the bounded waits without hanging the device. */
 DHSA_API dhsa_status dhsa_selftest_timeout(void* workspace, int32_t limit_us, void* stream);
+
+/* ---- step 0 (optional): online variable-length chunking -------------------
+ * The On-Device page (Abstract, AI Summary) says that DHSA segments each
+ * sequence adaptively and online into variable-length chunks, and gives no
+ * rule.  This library's rule is a plain one, decided left to right as tokens
+ * arrive: with the current chunk of a sequence starting at token b, token t
+ * starts a new chunk when
+ *     t - b >= max_len, or
+ *     t - b >= min_len and sim(t) < threshold,
+ * sim(t) = (1/Hkv) * sum_g cos(k[t-1, g], k[t, g]), cos(x, y) = x.y/(|x||y|),
+ * and 1 when either key is zero (a zero key never breaks a chunk).  The first
+ * chunk starts at the sequence's first token; the last may be shorter than
+ * min_len.  threshold <= -1 gives fixed max_len chunks, threshold > 1 fixed
+ * min_len chunks (while no key is zero).  sim is computed in fp32; a
+ * decision on a sim within about d * 2^-23 of the threshold may differ from
+ * one taken in exact arithmetic.
+ * The outputs are the chunk_bounds / seq_chunk_ptr arrays of dhsa_problem. */
+#define DHSA_SEGMENT_MAX_LEN 65536
+typedef struct {
+  float threshold;  /* finite, or +-infinity */
+  int32_t min_len;  /* 1 <= min_len <= max_len */
+  int32_t max_len;  /* max_len <= DHSA_SEGMENT_MAX_LEN */
+} dhsa_segment_rule;
+
+/* Host only: the most chunks any key values can give, sum over sequences of
+ * ceil(L_b / min_len) (every chunk but a sequence's last has >= min_len
+ * tokens).  h_cu_seqlens: host [B+1]. */
+DHSA_API dhsa_status dhsa_segment_capacity(const int32_t* h_cu_seqlens, int32_t num_seqs, int32_t min_len,
+                                           int64_t* max_chunks);
+/* Workspace of dhsa_segment for T tokens: the status word plus two bitmaps of
+ * ceil(T/32) words. */
+DHSA_API dhsa_status dhsa_segment_workspace_size(int32_t total_tokens, size_t* bytes);
+/*   k              device [T, Hkv, d] in `dtype` (bf16 or fp32), 16-byte aligned,
+ *                  d in {64, 128, 256}
+ *   cu_seqlens     device [B+1]; h_cu_seqlens its host mirror (T = h_cu_seqlens[B])
+ *   chunk_bounds   device int32 [max_chunks + 1], written: entries 0..n
+ *   max_chunks     >= dhsa_segment_capacity(...)
+ *   seq_chunk_ptr  device int32 [B + 1], written
+ *   num_chunks     device int32 [1], written: n
+ * The caller reads n (and mirrors the arrays to the host) before building the
+ * dhsa_problem of the later steps. */
+DHSA_API dhsa_status dhsa_segment(const void* k, int32_t dtype, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t num_seqs, const int32_t* cu_seqlens, const int32_t* h_cu_seqlens,
+                                  dhsa_segment_rule rule, int32_t* chunk_bounds, int64_t max_chunks,
+                                  int32_t* seq_chunk_ptr, int32_t* num_chunks, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* ---- steps 1-3 without a caller workspace ----------------------------------
  * No counterpart in the paper: an interface addition for callers that cannot

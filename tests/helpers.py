@@ -99,3 +99,66 @@ def attention_gate(got, want, dtype):
              float(np.linalg.norm(g - want) / max(np.linalg.norm(want), 1e-30)))
     assert np.all(err <= tol), ("attention error above gate", stats, float((err - tol).max()))
     return stats
+
+
+def segment_tie_band(head_dim):
+    """Half-width of the band around the threshold inside which an fp32
+    adjacent-key similarity may decide differently from the exact one: the
+    dot product and both squared norms of d terms accumulate at most about
+    d rounding errors of 2^-24 relative to |x||y| each, the square roots and
+    the division a few more, and the mean over heads one per head (bounded by
+    the 16 added), all doubled for margin."""
+    return (2 * head_dim + 16) * 2.0 ** -24
+
+
+def check_segmentation(bounds, seq_ptr, sim, cu_seqlens, rule, band):
+    """Checks a segmentation (from the GPU) against the exact similarities.
+
+    Every chunk must be a legal step of the rule, where a similarity within
+    ``band`` of the threshold may be taken either way.  Returns, per sequence,
+    the start of the first chunk whose step needed that latitude (None when no
+    step did): up to there the segmentation must be the exact rule's."""
+    bounds = np.asarray(bounds, dtype=np.int64)
+    ptr = np.asarray(seq_ptr, dtype=np.int64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    thr, lo, hi = float(rule.threshold), int(rule.min_len), int(rule.max_len)
+    sure = sim < thr - band     # a break is due
+    maybe = np.abs(sim - thr) <= band
+    assert ptr.shape[0] == cu.shape[0] and ptr[0] == 0 and ptr[-1] == bounds.shape[0] - 1
+    assert bounds[-1] == cu[-1]
+    first_loose = []
+    for s in range(cu.shape[0] - 1):
+        s0, s1 = int(cu[s]), int(cu[s + 1])
+        starts = bounds[ptr[s]:ptr[s + 1]].tolist()
+        first_loose.append(None)
+        if s1 == s0:
+            assert starts == []
+            continue
+        assert starts and starts[0] == s0, (s, starts[:3])
+        ends = starts[1:] + [s1]
+        for b, e in zip(starts, ends):
+            assert b < e <= s1 and e - b <= hi, (b, e)
+            inner = range(b + lo, min(e, b + hi))
+            assert not any(sure[t] for t in inner), ("missed break", b, e)
+            used = any(maybe[t] for t in inner)
+            if e < s1:
+                assert e - b >= lo, (b, e)
+                if e - b != hi:
+                    assert sure[e] or maybe[e], ("break without cause", b, e, sim[e])
+                    used = used or bool(maybe[e])
+            if used and first_loose[-1] is None:
+                first_loose[-1] = b
+    return first_loose
+
+
+def segmentations_agree_until_latitude(got_bounds, got_ptr, want_bounds, want_ptr, first_loose):
+    """Per sequence, the chunk starts of both segmentations up to and including
+    the first step that had latitude (where both chose from the same start)."""
+    for s, fl in enumerate(first_loose):
+        g = list(got_bounds[got_ptr[s]:got_ptr[s + 1]])
+        w = list(want_bounds[want_ptr[s]:want_ptr[s + 1]])
+        if fl is None:
+            assert g == w, s
+        else:
+            cut = g.index(fl) + 1
+            assert g[:cut] == w[:cut], s
