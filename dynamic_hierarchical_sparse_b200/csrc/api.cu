@@ -159,7 +159,8 @@ dhsa_status run_attention(const void* q, const void* k, const void* v, const dhs
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DHSA_ERR_INVALID_ARG;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf(static_cast<float>(p->head_dim));
   uint32_t* status = static_cast<uint32_t*>(workspace);
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  // status word, then the persistent attention kernel's work-item counter
+  if (cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
   if (p->dtype == DHSA_F32) {
     return cuda_status(launch_attention_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                             static_cast<const float*>(v), p->chunk_bounds, p->num_chunks, row_ptr,

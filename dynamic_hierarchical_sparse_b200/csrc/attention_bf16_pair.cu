@@ -73,8 +73,10 @@ constexpr bool kSplitP = true;
 constexpr bool kPackedF32 = true;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kSchedWarp = 11;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kRangeCap = 128;  // runs cached in shared memory; more continue from the plan
+constexpr int kRangeCap = 96;  // runs cached per item slot in shared memory; more continue from the plan
+constexpr int kItemUsers = 11;  // item-slot releases: producer, two MMA threads, eight softmax warps
 constexpr int kVStages = 3;     // V ring depth (K uses 2)
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -87,8 +89,9 @@ struct PairCfg {
   static constexpr int kOffQ = 0;  // tile a at kOffQ + a * kQBytes
   static constexpr int kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffRanges = kOffV + kVStages * kKVBytes;
-  static constexpr int kOffBar = kOffRanges + kRangeCap * 8;
+  static constexpr int kOffRanges = kOffV + kVStages * kKVBytes;  // two item slots
+  static constexpr int kOffItems = kOffRanges + 2 * kRangeCap * 8;  // two item descriptors
+  static constexpr int kOffBar = kOffItems + 2 * 64;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
   static constexpr uint32_t kColS = 0;    // + 128 a
   static constexpr uint32_t kColO = 256;  // + D a
@@ -107,8 +110,29 @@ enum {
   kBarPHalf = 16,   // + query tile: first 64 keys of P written
   kBarDrain = 18,   // + query tile
   kBarTurn = 20,    // + query tile: that tile's MMA thread ended a turn
-  kNumBars = 22
+  kBarQFree = 22,   // both MMA threads' last S of the item done: Q may be reloaded
+  kBarItemReady = 23,  // + slot: the scheduler wrote the slot's next item
+  kBarItemFree = 25,   // + slot: every role is done with the slot's item
+  kNumBars = 27
 };
+
+// One work item (a CTA's unit of work before it became persistent): query
+// chunk ci, one or two 128-row query tiles, their key tiles.  Written by the
+// scheduler warp into one of two slots, with the slot's run list.
+struct Item {
+  int done;  // 1: no work left
+  int ci;
+  int h, h1;  // heads of query tile 0 and tile 1
+  int q0_0, q0_1, q_end0, q_end1;
+  int valid1;
+  int cap;     // last key + 1 of the item's diagonal run
+  int p1;      // end of the plan row
+  int resume;  // plan position where the runs past the cached list continue
+  int ncached;
+  int nt, nt0;  // key tiles of the item, and the prefix of them that tile 0 takes
+  int pad;
+};
+static_assert(sizeof(Item) == 64, "item slot size");
 
 // Key tiles of one work item: cached runs first, then (if the run list
 // overflowed) runs merged on the fly from the plan in global memory.
@@ -232,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                           const int* __restrict__ bounds, const int* __restrict__ row_ptr,
                           const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
-                          int plan_group, int head_pair, float scale_log2, uint32_t* status) {
+                          int plan_group, int head_pair, int tiles, int total_items, float scale_log2,
+                          uint32_t* status, int* item_counter) {
   using C = PairCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -240,28 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::kOffBar;
   auto bar = [&](int idx) { return bar0 + 8u * static_cast<uint32_t>(idx); };
-  int2* ranges = reinterpret_cast<int2*>(smem + C::kOffRanges);
+  int2* ranges_all = reinterpret_cast<int2*>(smem + C::kOffRanges);
+  Item* items = reinterpret_cast<Item*>(smem + C::kOffItems);
   int* misc = reinterpret_cast<int*>(smem + C::kOffBar + 8 * kNumBars);
-  // misc[0] TMEM base, misc[1] abort flag, misc[2] cached runs, misc[3] resume position
+  // misc[0] TMEM base, misc[1] abort flag
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-
-  // Two query tiles per CTA: consecutive 128-row tiles of one head, or, with
-  // head_pair (a plan row per KV group, even group size), the same 128 rows of
-  // two heads 2m and 2m+1 of one group, which then share one key list.
-  const int ci = num_chunks - 1 - static_cast<int>(blockIdx.z);  // longest rows first
-  const int c_start = bounds[ci], c_end = bounds[ci + 1];
-  const int h = head_pair ? 2 * static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);  // tile 0's head
-  const int q0_0 = c_start + static_cast<int>(blockIdx.x) * (head_pair ? 1 : 2) * kBM;
-  if (q0_0 >= c_end) return;  // uniform: this chunk has fewer tiles
-  const int q0_1 = head_pair ? q0_0 : q0_0 + kBM;
-  const bool valid1 = head_pair || q0_1 < c_end;
-  const int q_end0 = min(q0_0 + kBM, c_end);
-  const int q_end1 = valid1 ? min(q0_1 + kBM, c_end) : q0_1;
-  const int cap = valid1 ? q_end1 : q_end0;
-  const int h1 = head_pair ? h + 1 : h;  // tile 1's head
-  const int g = h / group;
-  const int row_id = (h / plan_group) * num_chunks + ci;
-  const int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -272,47 +280,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarPFull + s), 4);  // one arrival per softmax warp
       mbar_init(bar(kBarOReady + s), 1);
       mbar_init(bar(kBarPHalf + s), 4);
-    }
-    for (int s = 0; s < kVStages; ++s) mbar_init(bar(kBarVFull + s), 1);
-    for (int s = 0; s < 4; ++s) mbar_init(bar(kBarRel + s), valid1 ? 2 : 1);  // one commit per MMA thread
-    for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarDrain + s), 1);
       mbar_init(bar(kBarTurn + s), 1);
+      mbar_init(bar(kBarItemReady + s), 1);
+      mbar_init(bar(kBarItemFree + s), kItemUsers);
     }
+    for (int s = 0; s < kVStages; ++s) mbar_init(bar(kBarVFull + s), 1);
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kBarRel + s), 2);  // one commit per MMA thread
+    mbar_init(bar(kBarQFree), 2);
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  if (warp == kProducerWarp) {
-    // merge the row's kept chunks into runs of consecutive chunks
-    if (lane == 0) misc[3] = p1;
-    __syncwarp();
-    int nstart = 0, nend = 0;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = p0; base < p1; base += 32) {
-      const int p = base + lane;
-      const bool valid = p < p1;
-      const int c = valid ? col[p] : 0;
-      int cprev = __shfl_up_sync(0xffffffffu, c, 1);
-      int cnext = __shfl_down_sync(0xffffffffu, c, 1);
-      if (lane == 0) cprev = (p > p0) ? col[p - 1] : -2;
-      if (lane == 31) cnext = (p + 1 < p1) ? col[p + 1] : -2;
-      const bool is_start = valid && (p == p0 || c != cprev + 1);
-      const bool is_end = valid && (p == p1 - 1 || cnext != c + 1);
-      const unsigned sm = __ballot_sync(0xffffffffu, is_start);
-      const unsigned em = __ballot_sync(0xffffffffu, is_end);
-      if (is_start) {
-        const int idx = nstart + __popc(sm & lt);
-        if (idx < kRangeCap) ranges[idx].x = bounds[c];
-        else if (idx == kRangeCap) misc[3] = p;
-      }
-      if (is_end) {
-        const int idx = nend + __popc(em & lt);
-        if (idx < kRangeCap) ranges[idx].y = bounds[c + 1];
-      }
-      nstart += __popc(sm);
-      nend += __popc(em);
-    }
-    if (lane == 0) misc[2] = min(nstart, kRangeCap);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(misc), kTmemCols);
@@ -322,87 +299,198 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
-  const int ncached = misc[2];
-  const int resume = misc[3];
 
-  // tile counts: all tiles (second query tile, or the only one) and the prefix of tile 0
-  int nt = 0, nt0 = 0;
-  {
-    TileWalk w;
-    w.init(ranges, ncached, col, bounds, resume, p1, cap);
-    int k0, ke;
-    while (w.next(k0, ke)) {
-      ++nt;
-      if (k0 < q_end0) ++nt0;
-    }
-  }
-  const int nt1 = valid1 ? nt : 0;
-
+  // Persistent: the CTA takes work items (query chunk, heads, pair of query
+  // tiles) from a global counter until none are left, in the order
+  // i = x + tiles * (y + H * z): chunk n-1-z (longest plan rows first), head
+  // (pair) y, tile pair x.  Every barrier phase and ring position below runs
+  // on across items, so one item's Q and K/V loads and first QK^T overlap the
+  // previous item's last softmax and epilogue.
   if (warp >= 8) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-  if (warp == kProducerWarp) {
-    if (lane == 0 && nt > 0) {
+  if (warp == kSchedWarp) {
+    // ------------------------------------------------------- scheduler
+    const int H = head_pair ? num_q_heads / 2 : num_q_heads;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int k = 0;; ++k) {
+      const int s = k & 1;
+      if (k >= 2 && !mbar_wait(bar(kBarItemFree + s), ((k - 2) >> 1) & 1, abort_flag, status)) break;
+      Item* d = items + s;
+      int2* ranges = ranges_all + s * kRangeCap;
+      // next non-empty item (chunks shorter than the longest have fewer tiles)
+      int ci = 0, hh = 0, q00 = 0, c_end = 0;
+      bool done = false;
+      while (true) {
+        int i = 0;
+        if (lane == 0) i = atomicAdd(item_counter, 1);
+        i = __shfl_sync(0xffffffffu, i, 0);
+        if (i >= total_items) {
+          done = true;
+          break;
+        }
+        const int x = i % tiles, r = i / tiles;
+        const int y = r % H, z = r / H;
+        ci = num_chunks - 1 - z;
+        const int c_start = bounds[ci];
+        c_end = bounds[ci + 1];
+        hh = head_pair ? 2 * y : y;
+        q00 = c_start + x * (head_pair ? 1 : 2) * kBM;
+        if (q00 < c_end) break;
+      }
+      if (done) {
+        if (lane == 0) d->done = 1;
+      } else {
+        // Two query tiles: consecutive 128-row tiles of one head, or, with
+        // head_pair (a plan row per KV group, even group size), the same 128
+        // rows of two heads 2m and 2m+1 of one group, sharing one key list.
+        const int q01 = head_pair ? q00 : q00 + kBM;
+        const bool valid1 = head_pair || q01 < c_end;
+        const int q_end0 = min(q00 + kBM, c_end);
+        const int q_end1 = valid1 ? min(q01 + kBM, c_end) : q01;
+        const int cap = valid1 ? q_end1 : q_end0;
+        const int row_id = (hh / plan_group) * num_chunks + ci;
+        const int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
+        // merge the row's kept chunks into runs of consecutive chunks
+        if (lane == 0) d->resume = p1;
+        __syncwarp();
+        int nstart = 0, nend = 0;
+        for (int base = p0; base < p1; base += 32) {
+          const int p = base + lane;
+          const bool valid = p < p1;
+          const int c = valid ? col[p] : 0;
+          int cprev = __shfl_up_sync(0xffffffffu, c, 1);
+          int cnext = __shfl_down_sync(0xffffffffu, c, 1);
+          if (lane == 0) cprev = (p > p0) ? col[p - 1] : -2;
+          if (lane == 31) cnext = (p + 1 < p1) ? col[p + 1] : -2;
+          const bool is_start = valid && (p == p0 || c != cprev + 1);
+          const bool is_end = valid && (p == p1 - 1 || cnext != c + 1);
+          const unsigned sm = __ballot_sync(0xffffffffu, is_start);
+          const unsigned em = __ballot_sync(0xffffffffu, is_end);
+          if (is_start) {
+            const int idx = nstart + __popc(sm & lt);
+            if (idx < kRangeCap) ranges[idx].x = bounds[c];
+            else if (idx == kRangeCap) d->resume = p;
+          }
+          if (is_end) {
+            const int idx = nend + __popc(em & lt);
+            if (idx < kRangeCap) ranges[idx].y = bounds[c + 1];
+          }
+          nstart += __popc(sm);
+          nend += __popc(em);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const int ncached = min(nstart, kRangeCap);
+          // key tiles of the item (tile 1, or the only tile) and tile 0's prefix
+          int nt = 0, nt0 = 0;
+          TileWalk w;
+          w.init(ranges, ncached, col, bounds, d->resume, p1, cap);
+          int k0, ke;
+          while (w.next(k0, ke)) {
+            ++nt;
+            if (k0 < q_end0) ++nt0;
+          }
+          d->done = 0;
+          d->ci = ci;
+          d->h = hh;
+          d->h1 = head_pair ? hh + 1 : hh;
+          d->q0_0 = q00;
+          d->q0_1 = q01;
+          d->q_end0 = q_end0;
+          d->q_end1 = q_end1;
+          d->valid1 = valid1 ? 1 : 0;
+          d->cap = cap;
+          d->p1 = p1;
+          d->ncached = ncached;
+          d->nt = nt;
+          d->nt0 = nt0;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarItemReady + s));
+      if (done) break;
+    }
+  } else if (warp == kProducerWarp) {
+    // -------------------------------------------------------- producer
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(kBarQ), (valid1 ? 2 : 1) * C::kQBytes);
-#pragma unroll
-      for (int a = 0; a < D / 64; ++a)
-        tma_load_3d(sbase + C::kOffQ + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h, q0_0);
-      if (valid1) {
+      int T = 0, issued = 0, qloads = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int s = k & 1;
+        if (!mbar_wait(bar(kBarItemReady + s), (k >> 1) & 1, abort_flag, status)) break;
+        const Item d = items[s];
+        if (d.done) break;
+        // Q of the previous item is free once both MMA threads' last S is done
+        if (k >= 1 && !mbar_wait(bar(kBarQFree), (k - 1) & 1, abort_flag, status)) break;
+        mbar_arrive_expect_tx(bar(kBarQ), (d.valid1 ? 2 : 1) * C::kQBytes);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a)
-          tma_load_3d(sbase + C::kOffQ + C::kQBytes + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h1, q0_1);
-      }
-      TileWalk w;
-      w.init(ranges, ncached, col, bounds, resume, p1, cap);
-      int k0, ke, issued = 0;
-      for (int t = 0; w.next(k0, ke); ++t) {
-        const int s = t & 1;
-        // K(t) replaces K(t-2), read by S(t-2); V(t) replaces V(t-3), read by
-        // PV(t-3), which was issued before S(t-2): both are free once the
-        // release commit that follows S(t-2) has landed.
-        if (t >= 2) {
-          const int j = t - 2;
-          if (!mbar_wait(bar(kBarRel + (j & 3)), (j >> 2) & 1, abort_flag, status)) break;
+          tma_load_3d(sbase + C::kOffQ + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, d.h, d.q0_0);
+        if (d.valid1) {
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(sbase + C::kOffQ + C::kQBytes + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, d.h1, d.q0_1);
         }
-        mbar_arrive_expect_tx(bar(kBarKFull + s), C::kKVBytes);
+        qloads = k + 1;
+        const int g = d.h / group;
+        TileWalk w;
+        w.init(ranges_all + s * kRangeCap, d.ncached, col, bounds, d.resume, d.p1, d.cap);
+        int k0, ke;
+        for (int t = 0; w.next(k0, ke); ++t) {
+          const int tg = T + t;  // key tile counted across items
+          const int st = tg & 1;
+          // K(tg) replaces K(tg-2), read by S(tg-2); V(tg) replaces V(tg-3),
+          // read by PV(tg-3), which each MMA thread issued before S(tg-2):
+          // both are free once the release commits that follow S(tg-2) land.
+          if (tg >= 2 && !mbar_wait(bar(kBarRel + ((tg - 2) & 3)), ((tg - 2) >> 2) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(kBarKFull + st), C::kKVBytes);
 #pragma unroll
-        for (int a = 0; a < D / 64; ++a)
-          tma_load_3d(sbase + C::kOffK + s * C::kKVBytes + a * C::kKVSub, &tm_k, bar(kBarKFull + s), a * 64, g, k0);
-        const int sv = t % kVStages;
-        mbar_arrive_expect_tx(bar(kBarVFull + sv), C::kKVBytes);
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(sbase + C::kOffK + st * C::kKVBytes + a * C::kKVSub, &tm_k, bar(kBarKFull + st), a * 64, g,
+                        k0);
+          const int sv = tg % kVStages;
+          mbar_arrive_expect_tx(bar(kBarVFull + sv), C::kKVBytes);
 #pragma unroll
-        for (int a = 0; a < D / 64; ++a)
-          tma_load_3d(sbase + C::kOffV + sv * C::kKVBytes + a * C::kKVSub, &tm_v, bar(kBarVFull + sv), a * 64, g,
-                      k0);
-        issued = t + 1;
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(sbase + C::kOffV + sv * C::kKVBytes + a * C::kKVSub, &tm_v, bar(kBarVFull + sv), a * 64, g,
+                        k0);
+          issued = tg + 1;
+        }
+        T += d.nt;
+        mbar_arrive(bar(kBarItemFree + s));
       }
       if (*abort_flag) {
         // let copies already in flight land before the CTA exits (bounded)
         volatile int never = 0;
-        mbar_wait(bar(kBarQ), 0, &never, nullptr, 10000000ull);
+        if (qloads > 0) mbar_wait(bar(kBarQ), (qloads - 1) & 1, &never, nullptr, 10000000ull);
         for (int t = max(0, issued - 2); t < issued; ++t)
           mbar_wait(bar(kBarKFull + (t & 1)), (t >> 1) & 1, &never, nullptr, 10000000ull);
         for (int t = max(0, issued - kVStages); t < issued; ++t)
           mbar_wait(bar(kBarVFull + t % kVStages), (t / kVStages) & 1, &never, nullptr, 10000000ull);
       }
     }
-  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+  } else {
+    // ----------------------------------------------------------- MMA
     // One MMA-issuing thread per query tile, taking turns: tile 0's thread
     // issues PV_0(t) and S_0(t+1), hands over, tile 1's thread issues PV_1(t)
     // and S_1(t+1), hands back.  The turns keep the two softmax warpgroups
     // half a period apart (so they do not share the exponential unit); two
     // threads let each one pass its own waits and commits while the other's
-    // MMAs run, instead of leaving the tensor pipe idle meanwhile.
+    // MMAs run, instead of leaving the tensor pipe idle meanwhile.  Both
+    // threads take every turn, also on items with one query tile.
     const int a = warp - kMmaWarp;
-    const int nta = a == 0 ? nt0 : nt1;
-    if (lane == 0 && nt > 0 && (a == 0 || valid1)) {
+    if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 1);
       const uint32_t qbase = sbase + C::kOffQ + a * C::kQBytes;
-      auto issue_s = [&](int t) {
-        const uint32_t kbase = sbase + C::kOffK + (t & 1) * C::kKVBytes;
+      auto issue_s = [&](int tg) {
+        const uint32_t kbase = sbase + C::kOffK + (tg & 1) * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(qbase + (kk >> 2) * C::kQSub + (kk & 3) * 32, 16, 1024);
@@ -411,58 +499,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(bar(kBarSFull + a));
       };
-      // turn k (0 = the first S, k = t + 1 for key tile t): tile 1's thread
-      // waits for tile 0's turn k, tile 0's thread for tile 1's turn k - 1
-      auto wait_turn = [&](int k) -> bool {
-        if (!valid1) return true;
-        if (a == 1) return mbar_wait_spin(bar(kBarTurn + 0), k & 1, abort_flag, status);
-        if (k == 0) return true;
-        return mbar_wait_spin(bar(kBarTurn + 1), (k - 1) & 1, abort_flag, status);
+      // turn kt (counted across items): tile 1's thread waits for tile 0's
+      // turn kt, tile 0's thread for tile 1's turn kt - 1
+      auto wait_turn = [&](int kt) -> bool {
+        if (a == 1) return mbar_wait_spin(bar(kBarTurn + 0), kt & 1, abort_flag, status);
+        if (kt == 0) return true;
+        return mbar_wait_spin(bar(kBarTurn + 1), (kt - 1) & 1, abort_flag, status);
       };
-      auto end_turn = [&]() {
-        if (valid1) mbar_arrive(bar(kBarTurn + a));
-      };
-      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, status);
-      if (ok) ok = mbar_wait(bar(kBarKFull + 0), 0, abort_flag, status);
-      if (ok) ok = wait_turn(0);
-      if (ok) {
+      auto end_turn = [&]() { mbar_arrive(bar(kBarTurn + a)); };
+      int T = 0, kt = 0, np = 0;  // key tiles, turns, P tiles of this query tile: all across items
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int s = k & 1;
+        if (!mbar_wait(bar(kBarItemReady + s), (k >> 1) & 1, abort_flag, status)) break;
+        const Item d = items[s];
+        if (d.done) break;
+        const int nt = d.nt;
+        const int nta = a == 0 ? d.nt0 : (d.valid1 ? d.nt : 0);
+        ok = mbar_wait(bar(kBarQ), k & 1, abort_flag, status);
+        if (ok) ok = mbar_wait(bar(kBarKFull + (T & 1)), (T >> 1) & 1, abort_flag, status);
+        if (ok) ok = wait_turn(kt);
+        if (!ok) break;
         tc_fence_after();
-        if (nta > 0) issue_s(0);
-        umma_commit(bar(kBarRel + 0));  // j = 0: S(0) done
+        if (nta > 0) issue_s(T);
+        if (nta <= 1) umma_commit(bar(kBarQFree));  // this thread's last S of the item (if any) is issued
+        umma_commit(bar(kBarRel + (T & 3)));         // key tile T: S(T) done
         end_turn();
-      }
-      for (int t = 0; ok && t < nt; ++t) {
-        const int sv = t % kVStages;
-        if (!mbar_wait_spin(bar(kBarVFull + sv), (t / kVStages) & 1, abort_flag, status)) break;
-        if (t < nta) {
-          const uint32_t vbase = sbase + C::kOffV + sv * C::kKVBytes;
-          auto issue_pv = [&](int kk0, int kk1) {
+        ++kt;
+        for (int t = 0; t < nt; ++t) {
+          const int tg = T + t;
+          if (t < nta) {
+            const int sv = tg % kVStages;
+            if (!mbar_wait_spin(bar(kBarVFull + sv), (tg / kVStages) & 1, abort_flag, status)) { ok = false; break; }
+            const uint32_t vbase = sbase + C::kOffV + sv * C::kKVBytes;
+            auto issue_pv = [&](int kk0, int kk1) {
 #pragma unroll
-            for (int kk = kk0; kk < kk1; ++kk) {
-              const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, C::kKVSub, 1024);
-              umma_f16_ts(tmem + C::kColO + a * D, tmem + C::kColS + a * 128 + kk * 8, bd, idesc_o,
-                          (t > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = kk0; kk < kk1; ++kk) {
+                const uint64_t bd = smem_desc_sw128(vbase + kk * 16 * 128, C::kKVSub, 1024);
+                umma_f16_ts(tmem + C::kColO + a * D, tmem + C::kColS + a * 128 + kk * 8, bd, idesc_o,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+              }
+            };
+            if (!mbar_wait_spin(bar(kBarPHalf + a), np & 1, abort_flag, status)) { ok = false; break; }
+            if (t + 1 < nta &&
+                !mbar_wait_spin(bar(kBarKFull + ((tg + 1) & 1)), ((tg + 1) >> 1) & 1, abort_flag, status)) {
+              ok = false;
+              break;
             }
-          };
-          if (!mbar_wait_spin(bar(kBarPHalf + a), t & 1, abort_flag, status)) break;
-          if (t + 1 < nta &&
-              !mbar_wait_spin(bar(kBarKFull + ((t + 1) & 1)), ((t + 1) >> 1) & 1, abort_flag, status))
+            if (!wait_turn(kt)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(0, kBN / 32);
+            if (!mbar_wait_spin(bar(kBarPFull + a), np & 1, abort_flag, status)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(kBN / 32, kBN / 16);
+            ++np;
+            // only the epilogue waits for O: S(t+1), issued after PV(t), tells
+            // the softmax that PV(t) is done before it rescales O
+            if (t + 1 == nta) umma_commit(bar(kBarOReady + a));
+            if (t + 1 < nta) {
+              issue_s(tg + 1);
+              if (t + 2 == nta) umma_commit(bar(kBarQFree));
+            }
+          } else if (!wait_turn(kt)) {
+            ok = false;
             break;
-          if (!wait_turn(t + 1)) break;
-          tc_fence_after();
-          issue_pv(0, kBN / 32);
-          if (!mbar_wait_spin(bar(kBarPFull + a), t & 1, abort_flag, status)) break;
-          tc_fence_after();
-          issue_pv(kBN / 32, kBN / 16);
-          // only the epilogue waits for O: S(t+1), issued after PV(t), tells
-          // the softmax that PV(t) is done before it rescales O
-          if (t + 1 == nta) umma_commit(bar(kBarOReady + a));
-          if (t + 1 < nta) issue_s(t + 1);
-        } else if (!wait_turn(t + 1)) {
-          break;
+          }
+          if (t + 1 < nt) umma_commit(bar(kBarRel + ((tg + 1) & 3)));  // key tile tg + 1: S(tg+1) done
+          end_turn();
+          ++kt;
         }
-        if (t + 1 < nt) umma_commit(bar(kBarRel + ((t + 1) & 3)));  // j = t + 1: S(t+1) done
-        end_turn();
+        T += nt;
+        mbar_arrive(bar(kBarItemFree + s));
       }
       // every MMA issued above completes before TMEM is released
       umma_commit(bar(kBarDrain + a));
@@ -474,25 +581,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------ softmax warpgroups
     const int a = warp >> 2;  // query tile of this warpgroup
-    const int nta = a == 0 ? nt0 : nt1;
-    const int q0 = a == 0 ? q0_0 : q0_1;
-    const int q_end = a == 0 ? q_end0 : q_end1;
     const int row = threadIdx.x & 127;
-    const int t_row = q0 + row;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + C::kColS + a * 128;
     const uint32_t tO = tmem + lane_base + C::kColO + a * D;
+    int ns = 0, no = 0;  // S tiles and epilogues of this query tile, across items
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+    const int slot = k & 1;
+    if (!mbar_wait(bar(kBarItemReady + slot), (k >> 1) & 1, abort_flag, status)) break;
+    const Item d = items[slot];
+    if (d.done) break;
+    const int nta = a == 0 ? d.nt0 : (d.valid1 ? d.nt : 0);
+    const int q0 = a == 0 ? d.q0_0 : d.q0_1;
+    const int q_end = a == 0 ? d.q_end0 : d.q_end1;
+    const int t_row = q0 + row;
     float m_run = -INFINITY;  // running max of logits * scale * log2(e)
     float l_run = 0.f;
     TileWalk w;
-    w.init(ranges, ncached, col, bounds, resume, p1, cap);
+    w.init(ranges_all + slot * kRangeCap, d.ncached, col, bounds, d.resume, d.p1, d.cap);
     int k0, ke;
-    bool ok = true;
     for (int t = 0; t < nta && w.next(k0, ke); ++t) {
-      if (!mbar_wait(bar(kBarSFull + a), t & 1, abort_flag, status)) {
+      if (!mbar_wait(bar(kBarSFull + a), ns & 1, abort_flag, status)) {
         ok = false;
         break;
       }
+      ++ns;
       tc_fence_after();
       // S row -> registers in two halves: the second half is still loading
       // while the first half is masked and max-reduced.
@@ -630,11 +744,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + a));
     }
-    if (ok && nta > 0 && mbar_wait(bar(kBarOReady + a), 0, abort_flag, status)) {
+    // done with the slot's run list; the epilogue needs registers only
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(kBarItemFree + slot));
+    if (!ok) break;
+    if (nta > 0) {
+      if (!mbar_wait(bar(kBarOReady + a), no & 1, abort_flag, status)) break;
+      ++no;
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const bool valid = t_row < q_end;
-      __nv_bfloat16* orow = out + (static_cast<size_t>(t_row) * num_q_heads + (a == 0 ? h : h1)) * D;
+      __nv_bfloat16* orow = out + (static_cast<size_t>(t_row) * num_q_heads + (a == 0 ? d.h : d.h1)) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -653,6 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+    }
     }
   }
 
@@ -676,12 +797,22 @@ cudaError_t launch_attention_pair_dim(const AttnBf16Args& a, cudaStream_t stream
   // a plan row per KV group of even size: pair two heads of the group on the same rows
   const int head_pair = (a.plan_group >= 2 && a.plan_group % 2 == 0) ? 1 : 0;
   const int tiles = head_pair ? (a.max_chunk_len + kBM - 1) / kBM : (a.max_chunk_len + 2 * kBM - 1) / (2 * kBM);
-  dim3 grid(tiles, head_pair ? a.num_q_heads / 2 : a.num_q_heads, a.num_chunks);
+  const int heads = head_pair ? a.num_q_heads / 2 : a.num_q_heads;
+  const long long total = static_cast<long long>(tiles) * heads * a.num_chunks;
+  if (total <= 0) return cudaSuccess;
+  if (total > 0x7fffffffLL - 2 * 65536) return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  // one persistent CTA per SM (its shared memory and TMEM fill the SM)
+  const int grid = static_cast<int>(total < sms ? total : sms);
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
                                                   a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
-                                                  a.num_q_heads / a.num_kv_heads, a.plan_group, head_pair,
-                                                  scale_log2, a.status);
+                                                  a.num_q_heads / a.num_kv_heads, a.plan_group, head_pair, tiles,
+                                                  static_cast<int>(total), scale_log2, a.status,
+                                                  reinterpret_cast<int*>(a.status + 1));
   return cudaGetLastError();
 }
 
