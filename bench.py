@@ -517,6 +517,77 @@ def bench_segment_micro(args):
     print(json.dumps(res), flush=True)
 
 
+def bench_online_chunking(args):
+    """The whole layer with online chunking: each step segments the keys on the
+    device (dhsa_segment), reads the chunk count and boundaries back to build
+    the problem on the host (the later steps size their launches from them),
+    then plans and attends.  128K LLaMA shape; the keys carry planted segments
+    U[256, 1024] (the default workload's chunk lengths), Q and V are the default
+    workload's.  Device-timed with CUDA events around whole steps, so the
+    host round trip is inside the timed region."""
+    from dynamic_hierarchical_sparse_b200 import api
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    spec = W.LLAMA_128K
+    inp = W.generate(spec, seed=0)
+    T = spec.total_tokens
+    k_host, cu, planted, planted_ptr = W.planted_segment_keys(0, [T], spec.num_kv_heads, spec.head_dim, 256, 1024)
+    rule = W.SegmentRule(0.5, 256, 1024)
+    q, k, v = inp.q.to(dev), k_host.to(dev), inp.v.to(dev)
+    out = torch.empty_like(q)
+    seg = api.Segmenter(cu, spec.num_kv_heads, spec.head_dim, rule, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        b, p, n = seg(k)
+        nh = int(n.item())  # waits for the segmentation
+        hb = b[:nh + 1].cpu().numpy()
+        hp = p.cpu().numpy()
+        if ev is not None:
+            ev[1].record(stream)
+        prob = api.Problem(cu, hb, hp, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, q.dtype, dev)
+        plan = api.Planner(prob, inp.budget, dev)(q, k)
+        if ev is not None:
+            ev[2].record(stream)
+        api.Attention(prob, dev)(q, k, v, plan, out)
+        if ev is not None:
+            ev[3].record(stream)
+        return hb, hp
+
+    for _ in range(args.warmup):
+        hb, hp = step()
+    torch.cuda.synchronize()
+    if seg.status() != 0:
+        raise RuntimeError("device-side status set during warm-up")
+    if not (np.array_equal(hb, planted) and np.array_equal(hp, planted_ptr)):
+        raise RuntimeError("online chunking did not recover the planted segments")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total = sum(e[0].elapsed_time(e[3]) for e in evs) / 1e3
+    part = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
+    print(json.dumps({
+        "metric": "DHSA prefill tokens/s at 128K with online chunking (1 B200)", "value": T * args.steps / total,
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (seeded; keys with planted segments U[256,1024])",
+        "config": {"workload": "llama31_8b_128k_h32kv8_d128_bf16_frac5 with online chunking",
+                   "rule": {"threshold": rule.threshold, "min_len": rule.min_len, "max_len": rule.max_len},
+                   "num_chunks": int(hb.shape[0] - 1), "budget": _budget_str(inp.budget)},
+        "ms_segment_and_readback": part[0], "ms_plan": part[1], "ms_attention": part[2],
+        "clocks": clk,
+    }), flush=True)
+
+
 def memory_report(spec, seed: int = 0, device=None):
     """Device memory of one DHSA layer call beyond its inputs and output.
 
@@ -620,6 +691,8 @@ def main():
     ap.add_argument("--memory", action="store_true", help="report device memory per layer call instead")
     ap.add_argument("--kv-plan", action="store_true",
                     help="grouped-query mode: one plan row per KV head (scored by the group's summed queries)")
+    ap.add_argument("--online-chunking", action="store_true",
+                    help="each step segments the keys online (dhsa_segment) before planning")
     ap.add_argument("--micro", default=None, choices=["select", "segment"],
                     help="time one kernel alone instead of the full step")
     args = ap.parse_args()
@@ -632,6 +705,8 @@ def main():
         bench_select_micro(args)
     elif args.micro == "segment":
         bench_segment_micro(args)
+    elif args.online_chunking:
+        bench_online_chunking(args)
     elif args.impl == "reference":
         bench_reference(args)
     else:
