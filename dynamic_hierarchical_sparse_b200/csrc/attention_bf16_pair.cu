@@ -1,6 +1,6 @@
 // Step 4 of the DHSA path for bf16 inputs, head_dim 64 and 128: varlen
 // block-sparse causal flash attention on tcgen05 tensor cores, two query tiles
-// per CTA.
+// per work item, one persistent CTA per SM.
 //
 // out[t, h] = sum_s softmax_s(q[t,h] . k[s,g] * scale) v[s,g] over the kept
 // key tokens s <= t: the tokens of the chunks in plan row (h, chunk(t))
@@ -9,25 +9,32 @@
 // upsampled chunk scores are preserved; "... for Memory-Constrained LLM
 // Inference": causally important dependencies are kept).
 //
-// Work item = one CTA = (query chunk i, head h, pair of 128-row tiles of chunk
-// i).  Both tiles walk the same key tiles, so every K/V tile brought into
-// shared memory by TMA feeds two QK^T and two PV products.  The kept chunks of
-// row (h, i) are merged into runs of consecutive chunks once per CTA (a list in
-// shared memory; rows with more runs than it holds continue from the plan in
-// global memory), each run is cut into 128-key tiles, and the run holding the
+// Work item = (query chunk i, head h, pair of 128-row tiles of chunk i).  Both
+// tiles walk the same key tiles, so every K/V tile brought into shared memory
+// by TMA feeds two QK^T and two PV products.  The kept chunks of row (h, i) are
+// merged into runs of consecutive chunks once per item (a list in shared
+// memory; rows with more runs than it holds continue from the plan in global
+// memory), each run is cut into 128-key tiles, and the run holding the
 // diagonal is clipped at the last valid query row of the pair.  The first tile
 // of the pair stops at its own last row, so its tiles are a prefix of the
 // second's.
 //
+// The kernel is persistent: one CTA per SM takes items from a counter in the
+// workspace until none are left, and every ring position and barrier phase
+// runs on across items, so an item's Q and K/V loads and its first QK^T
+// overlap the previous item's last softmax and epilogue.
+//
 // Warp roles (384 threads = three warpgroups):
 //   warps 0-3   softmax + epilogue of query tile 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of query tile 1
-//   warp 8      TMA producer: both Q tiles once, K tiles into a 2-stage ring,
-//               V tiles into a 3-stage ring; tile t+2 loads once the MMAs
+//   warp 8      TMA producer: both Q tiles of each item (once the previous
+//               item's last QK^T is done), K tiles into a 2-stage ring, V
+//               tiles into a 3-stage ring; tile t+2 loads once the MMAs
 //               through S(t) are done (one release commit per key tile)
 //   warp 9      TMEM allocator; its lane 0 issues the MMAs of query tile 0
 //   warp 10     lane 0 issues the MMAs of query tile 1
-//   warp 11     idle
+//   warp 11     scheduler: fetches the next item, builds its run list into the
+//               second of two item slots
 // The launch gives every thread 168 registers (three warps share a
 // sub-partition's 16K); the third warpgroup then hands registers back
 // (setmaxnreg.dec to 56) and the softmax warpgroups take them (224), enough to
