@@ -180,7 +180,10 @@ DHSA_API dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem*
  * accumulation and an fp32 online softmax; fp32 runs an fp32 kernel.
  *   q, k, v  device, THD, `dtype`; out device [T, Hq, d] in `dtype`
  *   row_ptr, col: a plan as written by dhsa_plan / dhsa_topk_select
- * Workspace: dhsa_attention_workspace_size bytes (status word + schedule). */
+ * Workspace: dhsa_attention_workspace_size bytes: the status word and the
+ * work-item counter of the persistent bf16 kernel, both reset by each call.
+ * A workspace serves one call at a time: calls that may overlap on the GPU
+ * (other streams) need workspaces of their own. */
 DHSA_API dhsa_status dhsa_attention_workspace_size(const dhsa_problem* p, size_t* bytes);
 DHSA_API dhsa_status dhsa_attention(const void* q, const void* k, const void* v,
                            const dhsa_problem* p, const int32_t* row_ptr,
