@@ -321,7 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const unsigned lt = (1u << lane) - 1u;
     for (int k = 0;; ++k) {
       const int s = k & 1;
-      if (k >= 2 && !mbar_wait(bar(kBarItemFree + s), ((k - 2) >> 1) & 1, abort_flag, status)) break;
+      // every lane waits; the warp leaves together if any lane gave up
+      const bool free_ok = k < 2 || mbar_wait(bar(kBarItemFree + s), ((k - 2) >> 1) & 1, abort_flag, status);
+      if (!__all_sync(0xffffffffu, free_ok)) break;
       Item* d = items + s;
       int2* ranges = ranges_all + s * kRangeCap;
       // next non-empty item (chunks shorter than the longest have fewer tiles)
