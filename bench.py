@@ -285,26 +285,30 @@ def bench_gpu(args):
 
     # ---------------- end to end through the public API with host buffers
     # Every step copies its Q/K/V in from pinned host memory and its output
-    # back out.  Two device buffer sets and three streams let step i's
+    # back out.  Three device buffer sets and three streams let step i's
     # copy-out, step i+1's copy-in and step i's plan + attention overlap (the
     # copies run in opposite directions over the host link), as a prefill
-    # server streaming requests would run them.
+    # server streaming requests would run them; with three sets a copy-in
+    # never waits for the copy-out of the step before.
+    nbuf = 3
     hq = inp.q.pin_memory()
     hk = inp.k.pin_memory()
     hv = inp.v.pin_memory()
-    houts = [torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory() for _ in range(2)]
-    dq, dk, dv = [q, torch.empty_like(q)], [k, torch.empty_like(k)], [v, torch.empty_like(v)]
-    douts = [out, torch.empty_like(out)]
+    houts = [torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory() for _ in range(nbuf)]
+    dq = [q] + [torch.empty_like(q) for _ in range(nbuf - 1)]
+    dk = [k] + [torch.empty_like(k) for _ in range(nbuf - 1)]
+    dv = [v] + [torch.empty_like(v) for _ in range(nbuf - 1)]
+    douts = [out] + [torch.empty_like(out) for _ in range(nbuf - 1)]
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    ev_in, ev_cmp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
-    e2e_steps = max(2, min(args.steps, 8))
+    ev_in, ev_cmp, ev_out = ([torch.cuda.Event() for _ in range(nbuf)] for _ in range(3))
+    e2e_steps = max(2, min(args.steps, 24))  # the stream's fill and drain amortised over up to 24 steps
 
     def e2e_run(nsteps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s_in)
         for i in range(nsteps):
-            b = i & 1
-            if i >= 2:  # buffer set b is free once step i-2's attention and copy-out are done
+            b = i % nbuf
+            if i >= nbuf:  # buffer set b is free once step i-nbuf's attention and copy-out are done
                 s_in.wait_event(ev_cmp[b])
                 s_in.wait_event(ev_out[b])
             with torch.cuda.stream(s_in):
@@ -368,7 +372,7 @@ def bench_gpu(args):
                 "steps": e2e_steps,
                 "schedule": "each step copies Q/K/V in from pinned host memory and O out; copy-in, "
                             "plan + attention and copy-out of consecutive steps overlap on three streams "
-                            "(two device buffer sets)"},
+                            "(three device buffer sets)"},
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
     }
