@@ -12,9 +12,9 @@
 //
 // Three launches:
 //  1. adjacent_sim_kernel: sim(t) for every token, four consecutive tokens per
-//     warp (each key row read once per warp, 16-byte vector loads, one squared
-//     norm per row), 32 tokens per CTA; one bit per token ("drop": sim(t) <
-//     threshold) into a bitmap.  HBM-bound: every key row is read once from
+//     warp (each key row read once per warp, 16-byte vector loads, up to two
+//     per lane and head, one squared norm per row), 32 tokens per CTA; one bit
+//     per token ("drop": sim(t) < threshold) into a bitmap.  HBM-bound: every key row is read once from
 //     DRAM (the row before a warp's first token, read by the neighbouring warp
 //     too, hits in cache).
 //  2. segment_walk_kernel: one CTA per sequence.  The sequence's drop bits are
@@ -58,20 +58,23 @@ __device__ __forceinline__ void to_float(const uint4& v, float* f, const float*)
 }
 
 // One warp takes R consecutive tokens tb .. tb+R-1 and reads each of the rows
-// tb-1 .. tb+R-1 once: every row's squared norm is formed once and feeds the
-// two cosines it takes part in.  Lanes form groups of G that cover one head's
-// vectors; P = 32 / G heads per pass over the heads.
+// tb-1 .. tb+R-1 once (all R+1 rows' loads are issued before any arithmetic):
+// every row's squared norm is formed once and feeds the two cosines it takes
+// part in.  A lane holds IT 16-byte vectors of one head (up to 2), so a head
+// is covered by G = V / IT lanes (a reduction of log2(G) shuffle steps) and a
+// pass over the heads takes P = 32 / G of them.
 template <typename T, int D>
 __global__ void __launch_bounds__(32 * kSimWarps)
     adjacent_sim_kernel(const T* __restrict__ k, int total_tokens, int hkv, float threshold,
                         uint32_t* __restrict__ drop, uint32_t* __restrict__ start_bits) {
   constexpr int E = 16 / static_cast<int>(sizeof(T));  // elements per 16-byte vector
   constexpr int V = D / E;                            // vectors per head
-  constexpr int G = V < 32 ? V : 32;                  // lanes per head
+  constexpr int IT = V < 2 ? V : 2;                   // vectors per lane per head
+  constexpr int G = V / IT;                           // lanes per head
   constexpr int P = 32 / G;                           // heads per pass
-  constexpr int IT = V / G;                           // vectors per lane per head
-  constexpr int F = IT * E;                           // floats per lane per row and pass
+  constexpr int F = IT * E;                           // floats per lane per row
   constexpr int R = 32 / kSimWarps;                   // tokens per warp
+  static_assert(G >= 1 && G <= 32 && (G & (G - 1)) == 0, "lanes per head");
   __shared__ uint32_t s_word;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * 32;
@@ -86,44 +89,43 @@ __global__ void __launch_bounds__(32 * kSimWarps)
   for (int g0 = 0; g0 < hkv; g0 += P) {
     const int g = g0 + lane / G;
     const bool on = g < hkv;
-    float x[R + 1][F];
+    uint4 raw[R + 1][IT];
 #pragma unroll
     for (int r = 0; r <= R; ++r) {
       const int t = tb - 1 + r;
       const bool valid = on && t >= 0 && t < total_tokens;
 #pragma unroll
-      for (int it = 0; it < IT; ++it) {
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (valid) u = __ldg(kv + static_cast<size_t>(t) * rowv + g * V + it * G + sub);
-        to_float(u, &x[r][it * E], static_cast<const T*>(nullptr));
-      }
+      for (int it = 0; it < IT; ++it)
+        raw[r][it] = valid ? __ldg(kv + static_cast<size_t>(t) * rowv + g * V + it * G + sub)
+                           : make_uint4(0u, 0u, 0u, 0u);
     }
-    float nrm[R + 1], dot[R];
+    float prev[F], cur[F];
 #pragma unroll
-    for (int r = 0; r <= R; ++r) {
-      float s = 0.f;
+    for (int it = 0; it < IT; ++it) to_float(raw[0][it], &prev[it * E], static_cast<const T*>(nullptr));
+    float nprev = 0.f;
 #pragma unroll
-      for (int e = 0; e < F; ++e) s = fmaf(x[r][e], x[r][e], s);
-      nrm[r] = s;
-    }
+    for (int e = 0; e < F; ++e) nprev = fmaf(prev[e], prev[e], nprev);
+#pragma unroll
+    for (int o = G / 2; o >= 1; o >>= 1) nprev += __shfl_xor_sync(0xffffffffu, nprev, o);
 #pragma unroll
     for (int j = 0; j < R; ++j) {
-      float s = 0.f;
 #pragma unroll
-      for (int e = 0; e < F; ++e) s = fmaf(x[j][e], x[j + 1][e], s);
-      dot[j] = s;
-    }
+      for (int it = 0; it < IT; ++it) to_float(raw[j + 1][it], &cur[it * E], static_cast<const T*>(nullptr));
+      float ncur = 0.f, dot = 0.f;
 #pragma unroll
-    for (int o = G / 2; o >= 1; o >>= 1) {
+      for (int e = 0; e < F; ++e) {
+        ncur = fmaf(cur[e], cur[e], ncur);
+        dot = fmaf(prev[e], cur[e], dot);
+      }
 #pragma unroll
-      for (int r = 0; r <= R; ++r) nrm[r] += __shfl_xor_sync(0xffffffffu, nrm[r], o);
+      for (int o = G / 2; o >= 1; o >>= 1) {
+        ncur += __shfl_xor_sync(0xffffffffu, ncur, o);
+        dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      }
+      if (sub == 0 && on) acc[j] += (nprev > 0.f && ncur > 0.f) ? dot * rsqrtf(nprev) * rsqrtf(ncur) : 1.f;
 #pragma unroll
-      for (int j = 0; j < R; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], o);
-    }
-    if (sub == 0 && on) {
-#pragma unroll
-      for (int j = 0; j < R; ++j)
-        acc[j] += (nrm[j] > 0.f && nrm[j + 1] > 0.f) ? dot[j] * rsqrtf(nrm[j]) * rsqrtf(nrm[j + 1]) : 1.f;
+      for (int e = 0; e < F; ++e) prev[e] = cur[e];
+      nprev = ncur;
     }
   }
 #pragma unroll
