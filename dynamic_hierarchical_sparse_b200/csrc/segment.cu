@@ -38,6 +38,7 @@ namespace {
 constexpr int kSimWarps = 8;             // warps per CTA; 32 tokens per CTA
 constexpr int kWinWords = 4096;          // walk window: 131072 tokens (max_len <= 65536)
 constexpr int kWalkThreads = 256;
+constexpr int kStartBuf = 1024;          // chunk starts the walking thread lists before the CTA writes them
 constexpr int kCompactThreads = 1024;
 
 __device__ __forceinline__ void to_float(const uint4& v, float* f, const __nv_bfloat16*) {
@@ -157,7 +158,8 @@ __global__ void __launch_bounds__(kWalkThreads)
   __shared__ int nd[kWinWords + 1];  // nd[i]: first drop at or after word wb + i (in the window), else kNone
   __shared__ int s_carry[kWalkThreads / 32];
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_abort, s_b, s_done;
+  __shared__ int s_starts[kStartBuf];  // chunk starts found by the walk, written out by the CTA
+  __shared__ int s_abort, s_b, s_done, s_nstarts;
   constexpr int kNone = 0x7fffffff;
   const int seq = blockIdx.x;
   const int s0 = cu_seqlens[seq], s1 = cu_seqlens[seq + 1];
@@ -222,15 +224,18 @@ __global__ void __launch_bounds__(kWalkThreads)
     }
     if (tid == 0) {
       // the walk: two shared-memory loads per chunk
-      int cb = b, done = 0;
-      while (true) {
+      int cb = b, done = 0, ns = 0;
+      while (ns < kStartBuf) {
         const int clo = cb + min_len;
         if (clo >= s1) { done = 1; break; }
         const int chi = min(cb + max_len, s1);
         const int wl = clo >> 5;
         if (((chi - 1) >> 5) >= wb + kWinWords) break;  // the window must move first
-        const uint32_t m = win[wl - wb] & (0xffffffffu << (clo & 31));
-        const int f = m != 0u ? (wl << 5) + __ffs(m) - 1 : nd[wl - wb + 1];
+        // both loads depend on wl only: issue them together
+        const uint32_t w = win[wl - wb];
+        const int beyond = nd[wl - wb + 1];
+        const uint32_t m = w & (0xffffffffu << (clo & 31));
+        const int f = m != 0u ? (wl << 5) + __ffs(m) - 1 : beyond;
         int next;
         if (f < chi) {
           next = f;
@@ -240,16 +245,21 @@ __global__ void __launch_bounds__(kWalkThreads)
           done = 1;
           break;
         }
-        atomicOr(start_bits + (next >> 5), 1u << (next & 31));
+        s_starts[ns++] = next;
         cb = next;
       }
       s_b = cb;
       s_done = done;
+      s_nstarts = ns;
     }
     __syncthreads();
     b = s_b;
     const int fin = s_done;
-    __syncthreads();  // s_b / s_done are rewritten by the next round
+    for (int i = tid; i < s_nstarts; i += kWalkThreads) {
+      const int p = s_starts[i];
+      atomicOr(start_bits + (p >> 5), 1u << (p & 31));
+    }
+    __syncthreads();  // s_b, s_done and the start list are rewritten by the next round
     if (fin) break;
   }
 }
