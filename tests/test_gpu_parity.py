@@ -276,6 +276,35 @@ def test_custom_scale_and_repeat_calls_are_deterministic():
     attention_gate(o1, want, torch.bfloat16)
 
 
+def test_concurrent_calls_on_two_streams():
+    """Attention calls overlapping on two streams, each with its own workspace
+    (status word and work-item counter of the persistent kernel), give the
+    outputs of the same calls run one after the other."""
+    cases = [_case("d128_long_runs"), _case("ragged_d128_top2")]
+    dev = torch.device("cuda")
+    runs = []
+    for inp in cases:
+        q, k, v, prob = to_device(inp)
+        plan = api.plan(q, k, prob, inp.budget, check=True)
+        runs.append((q, k, v, prob, plan, api.Attention(prob, dev)))
+    serial = []
+    for q, k, v, prob, plan, attn in runs:
+        out = torch.empty_like(q)
+        attn(q, k, v, plan, out)
+        serial.append(out)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.empty_like(r[0]) for r in runs]
+    for rep in range(3):
+        for (q, k, v, prob, plan, attn), out, st in zip(runs, outs, streams):
+            st.wait_stream(torch.cuda.current_stream())
+            attn(q, k, v, plan, out, stream=st)
+        torch.cuda.synchronize()
+        for (q, k, v, prob, plan, attn), out, ref, st in zip(runs, outs, serial, streams):
+            assert attn.status(st) == 0
+            assert torch.equal(out, ref), rep
+
+
 def test_empty_sequence_in_batch():
     inp = W.random_problem(7, [500, 0, 300], 2, 1, 64, "bf16", 40, 120, W.Budget.topk(2))
     q, k, v, prob = to_device(inp)
