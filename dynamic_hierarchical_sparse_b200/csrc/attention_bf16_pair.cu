@@ -531,10 +531,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         if (nta > 0) issue_s(T);
-        if (nta <= 1) umma_commit(bar(kBarQFree));  // this thread's last S of the item (if any) is issued
-        umma_commit(bar(kBarRel + (T & 3)));         // key tile T: S(T) done
+        // hand the turn over first: the other thread's MMAs wait for it, the
+        // commits below only for later consumers
         end_turn();
         ++kt;
+        if (nta <= 1) umma_commit(bar(kBarQFree));  // this thread's last S of the item (if any) is issued
+        umma_commit(bar(kBarRel + (T & 3)));         // key tile T: S(T) done
         for (int t = 0; t < nt; ++t) {
           const int tg = T + t;
           if (t < nta) {
@@ -562,20 +564,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             issue_pv(kBN / 32, kBN / 16);
             ++np;
+            if (t + 1 < nta) issue_s(tg + 1);
+            end_turn();
+            ++kt;
             // only the epilogue waits for O: S(t+1), issued after PV(t), tells
             // the softmax that PV(t) is done before it rescales O
             if (t + 1 == nta) umma_commit(bar(kBarOReady + a));
-            if (t + 1 < nta) {
-              issue_s(tg + 1);
-              if (t + 2 == nta) umma_commit(bar(kBarQFree));
+            if (t + 2 == nta) umma_commit(bar(kBarQFree));  // S(t+1) was the item's last
+          } else {
+            if (!wait_turn(kt)) {
+              ok = false;
+              break;
             }
-          } else if (!wait_turn(kt)) {
-            ok = false;
-            break;
+            end_turn();
+            ++kt;
           }
           if (t + 1 < nt) umma_commit(bar(kBarRel + ((tg + 1) & 3)));  // key tile tg + 1: S(tg+1) done
-          end_turn();
-          ++kt;
         }
         T += nt;
         mbar_arrive(bar(kBarItemFree + s));
