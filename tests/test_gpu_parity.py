@@ -43,6 +43,13 @@ def _case(name):
         return W.random_problem(10, [2000], 4, 2, 128, "bf16", 96, 96, W.Budget.topk(3), "structured")
     if name == "d64_fixed256":
         return W.random_problem(11, [2048, 1024], 2, 1, 64, "bf16", 256, 256, W.Budget.fraction(1, 4))
+    if name == "d128_group3":
+        # three query heads per KV head: a per-KV-head plan cannot pair heads
+        return W.random_problem(12, [1700, 900], 6, 2, 128, "bf16", 60, 300, W.Budget.fraction(1, 4), "structured")
+    if name == "d64_group3":
+        return W.random_problem(13, [1300], 3, 1, 64, "bf16", 40, 200, W.Budget.topk(3))
+    if name == "d256_group3":
+        return W.random_problem(14, [1200], 3, 1, 256, "bf16", 64, 256, W.Budget.topk(2), "structured")
     if name == "tiny_f32":
         return W.generate(W.TINY_1K_F32, 0)
     if name == "f32_d128_ragged":
@@ -52,7 +59,7 @@ def _case(name):
 
 CASES = ["ragged_d128_top2", "ragged_d64_frac", "d256_structured_top3", "d128_dense", "d128_diag_only",
          "d128_long_runs", "d128_many_runs", "d64_many_runs", "d128_fixed96", "d64_fixed256", "tiny_f32",
-         "f32_d128_ragged"]
+         "f32_d128_ragged", "d128_group3"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -223,7 +230,7 @@ def test_plan_and_attention(name):
 
 
 @pytest.mark.parametrize("name", ["ragged_d128_top2", "ragged_d64_frac", "d256_structured_top3", "d128_many_runs",
-                                  "d128_fixed96", "f32_d128_ragged"])
+                                  "d128_fixed96", "f32_d128_ragged", "d128_group3", "d64_group3", "d256_group3"])
 def test_per_kv_head_plan_and_attention(name):
     """Grouped-query mode: one plan row per KV head, scored by the group's
     summed query chunks, equals the oracle's per-KV-head plan (near-tie rule),
