@@ -43,7 +43,7 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # launch at the default 128K workload (9.43 GB + 1.04 GB), from a one-pass ncu
 # capture of the current kernel (profiles/attention_pair_llama128k_dram.md).
 # Must be reset to None whenever that kernel changes.
-ATTN_TRAFFIC_BYTES_PER_LAUNCH = 10.47e9
+ATTN_TRAFFIC_BYTES_PER_LAUNCH = None  # re-measured below
 
 
 def _peaks():

@@ -234,6 +234,12 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   return r;
 }
 
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -712,16 +718,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O is rescaled before PV(t) accumulates into it; PV(t-1) is done, since
       // S(t), waited for above, was issued after it
+      // two 32-column slices per round: both loads in flight, one wait, packed
+      // multiplies, both stores (the next round's loads touch other columns)
       auto rescale_o = [&]() -> bool {
+        const uint64_t alpha2 = f2_pack(alpha, alpha);
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
+        for (int c = 0; c < D / 32; c += 2) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tO + 32 * c, o0);
+          tmem_ld32(tO + 32 * (c + 1), o1);
           tmem_wait_ld();
-          reg_dep32(o);
+          reg_dep32(o0);
+          reg_dep32(o1);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + 32 * c, o);
+          for (int e = 0; e < 32; e += 2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o0[e]), __uint_as_float(o0[e + 1])), alpha2), x0, x1);
+            o0[e] = __float_as_uint(x0);
+            o0[e + 1] = __float_as_uint(x1);
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o1[e]), __uint_as_float(o1[e + 1])), alpha2), x0, x1);
+            o1[e] = __float_as_uint(x0);
+            o1[e + 1] = __float_as_uint(x1);
+          }
+          tmem_st32(tO + 32 * c, o0);
+          tmem_st32(tO + 32 * (c + 1), o1);
         }
         return true;
       };
