@@ -40,10 +40,10 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = W.LLAMA_128K.name
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention_pair_kernel<128>
-# launch at the default 128K workload (9.43 GB + 1.04 GB), from a one-pass ncu
+# launch at the default 128K workload (9.40 GB + 1.04 GB), from a one-pass ncu
 # capture of the current kernel (profiles/attention_pair_llama128k_dram.md).
 # Must be reset to None whenever that kernel changes.
-ATTN_TRAFFIC_BYTES_PER_LAUNCH = None  # re-measured below
+ATTN_TRAFFIC_BYTES_PER_LAUNCH = 10.44e9
 
 
 def _peaks():
