@@ -48,13 +48,17 @@
 // over): the pipe queues about one MMA, so a lone issuing thread runs in lock
 // step with it and its own barrier waits and commits between bursts would
 // leave the pipe idle; with two, each passes its waits during the other's
-// turn.  The P barriers take one arrival per softmax warp.
+// turn.  A thread hands the turn over right after its last MMA of the turn
+// (and the S-ready commit its own softmax waits for); the release, Q-free and
+// O-ready commits, which only later consumers wait for, come after.  The P
+// barriers take one arrival per softmax warp.
 // P reaches the tensor core in two halves of 64 keys, each behind its own
 // barrier, so PV_a(t) on the first half runs while the second half is still
 // being exponentiated.
 // Online softmax in fp32, exp2 domain, one ex2.approx per element (the
 // scale-and-shift and the row sums on packed f32x2 FMA / add), lazy O rescale
-// (only when a warp's running max grows by more than 2^8).
+// (only when a warp's running max grows by more than 2^8; two rounds of two
+// 32-column TMEM slices with packed multiplies).
 #include "common.cuh"
 #include "exp2_poly.cuh"
 #include "launchers.h"
