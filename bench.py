@@ -45,6 +45,9 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # Must be reset to None whenever that kernel changes.
 ATTN_TRAFFIC_BYTES_PER_LAUNCH = 10.44e9
 
+# FP32 FFMA ceiling of one B200: 148 SMs x 128 FP32 lanes x 2 FLOP per FMA x 1965 MHz
+FP32_FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -341,7 +344,15 @@ def bench_gpu(args):
 
     peaks = _peaks()
     achieved_tflops = flops_attn / t_attn / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    if spec.dtype == "bf16":
+        kernel = ("attention_pair_kernel<%d>" % spec.head_dim if spec.head_dim in (64, 128)
+                  else "attention_bf16_kernel<%d,64>" % spec.head_dim)
+        bound, peak = "tensor", peaks["bf16_tflops_sustained"]
+        peak_kind = "%s bf16 dense, sustained (kernel timed inside a seconds-long loop)" % peaks["source"]
+    else:
+        # fp32 inputs run the FFMA kernel: its ceiling is the FP32 pipe, not the tensor cores
+        kernel, bound, peak = "attention_f32_kernel<%d>" % spec.head_dim, "alu", FP32_FFMA_TFLOPS
+        peak_kind = "nominal fp32 FFMA: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz"
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_elapsed / args.steps * 1e3, "higher_is_better": True,
@@ -360,11 +371,8 @@ def bench_gpu(args):
         "t_plan_ms": t_plan * 1e3, "t_attn_ms": t_attn * 1e3,
         "plan_hbm_gbs": reduce_bytes / t_plan / 1e9,
         "roofline": {
-            "kernel": "attention_pair_kernel<%d>" % spec.head_dim if spec.head_dim in (64, 128)
-                      else "attention_bf16_kernel<%d,64>" % spec.head_dim,
-            "bound": "tensor", "achieved": achieved_tflops,
-            "peak": peak, "unit": "TFLOP/s", "frac": achieved_tflops / peak,
-            "peak_kind": "%s bf16 dense, sustained (kernel timed inside a seconds-long loop)" % peaks["source"],
+            "kernel": kernel, "bound": bound, "achieved": achieved_tflops,
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved_tflops / peak, "peak_kind": peak_kind,
             "traffic": ATTN_TRAFFIC_BYTES_PER_LAUNCH if spec.name == DEFAULT_WORKLOAD and not args.kv_plan else None,
             "algorithmic_flops_per_launch": flops_attn,
         },
