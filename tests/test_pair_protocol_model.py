@@ -80,3 +80,26 @@ def test_barrier_flags_a_waiter_two_phases_behind():
     b.arrive("x", 0, _Waiters())
     with pytest.raises(M.ProtocolViolation):
         b.arrive("x", 1, _Waiters([("late", 0)]))  # phase 1 completes while a waiter still waits for phase 0
+
+
+def test_model_constants_match_the_kernel_source():
+    """The barrier arrival counts and ring depths the model assumes are the ones
+    the kernel initialises (guards the model against drifting from the source)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "dynamic_hierarchical_sparse_b200", "csrc",
+                            "attention_bf16_pair.cu")).read()
+    consts = dict(re.findall(r"constexpr int (k\w+) = (\d+);", src))
+    assert int(consts["kVStages"]) == M.V_STAGES
+    assert int(consts["kItemUsers"]) == M.ITEM_USERS
+    counts = {}
+    for name, count in re.findall(r"mbar_init\(bar\((kBar\w+)(?: \+ s)?\), (\w+)\)", src):
+        counts[name] = int(consts.get(count, count))
+    model = M.Model([M.ItemSpec(1, 1, False)])
+    want = {"kBarQ": "Q", "kBarKFull": "KFull0", "kBarVFull": "VFull0", "kBarRel": "Rel0", "kBarSFull": "SFull0",
+            "kBarPFull": "PFull0", "kBarPHalf": "PHalf0", "kBarOReady": "OReady0", "kBarTurn": "Turn0",
+            "kBarQFree": "QFree", "kBarItemReady": "ItemReady0", "kBarItemFree": "ItemFree0"}
+    for kname, mname in want.items():
+        assert counts[kname] == model.bars[mname].count, kname
+    assert re.search(r"for \(int s = 0; s < %d; \+\+s\) mbar_init\(bar\(kBarRel \+ s\)" % M.REL_SLOTS, src)
+    assert "kOffV = kOffK + %d * kKVBytes" % M.K_STAGES in src
