@@ -479,6 +479,14 @@ class Model:
         """Runs to completion under a random schedule; returns the step count.
         Raises ProtocolViolation on a broken invariant or a deadlock."""
         rng = self.rng
+        # each actor runs at its own random speed (log-uniform over four decades),
+        # so that schedules where one role lags far behind the others are common
+        weight: Dict[tuple, float] = {}
+
+        def wt(key):
+            if key not in weight:
+                weight[key] = 10.0 ** rng.uniform(-4.0, 0.0)
+            return weight[key]
         for step in range(max_steps):
             choices = []
             for r in self.roles:
@@ -500,7 +508,8 @@ class Model:
                     return step
                 stuck = {r: self.pending_op[r] for r in self.roles if r not in self.finished}
                 raise ProtocolViolation("deadlock: %s" % stuck)
-            kind, x = choices[rng.randrange(len(choices))]
+            keys = [(c[0], c[1] if c[0] != "tma" else self.tma[c[1]][0]) for c in choices]
+            kind, x = rng.choices(choices, weights=[wt(key) for key in keys])[0]
             if kind == "tma":
                 self._land_tma(x)
             elif kind == "mma":
