@@ -2,8 +2,8 @@
 //
 // rep[h, c, :] = (sum_{t in chunk c} x[t, h, :]) / sqrt(L_c)   ("Long-Context
 // Modeling with Dynamic Hierarchical Sparse Attention for On-Device LLMs",
-// Abstract: chunk representations aggregate the chunk's token embeddings and
-// the average is scaled by the square root of the chunk size).
+// Abstract: a chunk is represented by the mean of its tokens' vectors,
+// multiplied by sqrt(L_c) to normalise for its length).
 //
 // HBM-bound streaming reduction.  One CTA owns one chunk and one 16-byte-per-
 // lane column slice of the token row (H*d elements): every warp reads whole

@@ -11,21 +11,21 @@ Hierarchical Sparse Attention for Memory-Constrained LLM Inference",
 abstract):
 
 1. ``chunk_representations``: each variable-length chunk is aggregated into one
-   vector by averaging its token embeddings and scaling the average by the
-   square root of the chunk length (length-normalised aggregation; On-Device
-   page, Abstract).  Mean times sqrt(L) equals sum divided by sqrt(L).
+   vector: the mean of its tokens' vectors times sqrt(L), L the chunk length
+   (length-normalised aggregation; On-Device page, Abstract).  Mean times
+   sqrt(L) equals sum divided by sqrt(L).
 2. ``chunk_scores``: chunk-level similarity is the dot product of a query-chunk
-   representation and a key-chunk representation (On-Device page, Abstract,
-   "chunk-level similarity scores").
+   representation and a key-chunk representation (On-Device page, Abstract:
+   similarity is scored between chunks).
 3. ``build_plan``: the chunk score is upsampled to token level (every token pair
    of chunks (i, j) inherits score(i, j)); for each query chunk the top-k
    causally admissible key chunks (earlier chunks of the same sequence) are kept
    by (score descending, chunk index ascending), and the diagonal chunk is kept
-   in addition (On-Device page, Abstract: "upsamples the chunk-level similarity
-   scores to token level similarities to calculate importance scores";
-   Memory-Constrained page, abstract: "estimating importance at the chunk level
-   and propagating it to token-level interactions, preserving causally important
-   dependencies").  Because every token of a chunk pair inherits one score,
+   in addition (On-Device page, Abstract: the chunk scores are carried down to
+   token level, where they act as the importance of each token interaction;
+   Memory-Constrained page, abstract: importance is judged per chunk, handed on
+   to the token interactions, and the causal dependencies that matter are
+   kept).  Because every token of a chunk pair inherits one score,
    selecting the best tokens by upsampled score keeps whole chunks;
    ``attention_literal`` re-derives the keep set from the materialised
    token-level score matrix to check that equivalence.
@@ -34,7 +34,7 @@ abstract):
    softmax attention of each query token over the kept key tokens only.
 
 Readings taken where the pages are silent (each listed in the design notes):
-per-head Q/K as the "token embeddings"; plain dot product without 1/sqrt(d);
+per-head Q/K as the per-token vectors that are aggregated; plain dot product without 1/sqrt(d);
 admissible key chunks are j < i in the same sequence, the diagonal is added on
 top of k; k above the admissible count keeps all; a fractional budget keeps
 ceil(i_local * num / den) chunks (integer arithmetic) capped at i_local; ties go
