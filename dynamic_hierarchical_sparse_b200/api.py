@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import dataclasses
 import os
+import threading
 from typing import Optional, Tuple
 
 import numpy as np
@@ -19,6 +20,7 @@ from .workloads import Budget
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdhsa.so")
 _lib = None
+_lib_lock = threading.Lock()
 
 DHSA_BF16 = 0
 DHSA_F32 = 1
@@ -71,7 +73,11 @@ def library_path() -> str:
 def lib() -> ctypes.CDLL:
     """The loaded library; raises if it has not been built."""
     global _lib
-    if _lib is None:
+    if _lib is not None:
+        return _lib
+    with _lib_lock:  # one thread loads the library and sets every signature
+        if _lib is not None:
+            return _lib
         if not os.path.exists(_LIB_PATH):
             raise RuntimeError("libdhsa.so is missing (build it with "
                                "`python -m dynamic_hierarchical_sparse_b200.build`)")

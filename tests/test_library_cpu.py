@@ -193,6 +193,25 @@ def test_product_path_has_no_cpu_fallback(monkeypatch):
         api.lib()
 
 
+def test_library_loads_once_under_concurrent_first_calls(monkeypatch):
+    """Threads racing on the first call all get the one loaded library, with
+    every signature set."""
+    import threading
+    monkeypatch.setattr(api, "_lib", None)
+    got, barrier = [], threading.Barrier(8)
+
+    def first_call():
+        barrier.wait()
+        got.append(api.lib())
+    threads = [threading.Thread(target=first_call) for _ in range(8)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert len(got) == 8 and all(g is got[0] for g in got)
+    assert got[0].dhsa_plan.argtypes is not None and got[0].dhsa_segment.restype is ctypes.c_int
+
+
 def test_product_package_does_not_import_the_oracle():
     pkg = os.path.join(ROOT, "dynamic_hierarchical_sparse_b200")
     pat = re.compile(r"^\s*(from\s+oracle|import\s+oracle)|dhsa_oracle", re.M)
