@@ -122,6 +122,20 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _enter(stream) -> None:
+    """A one-shot call on an explicit stream first waits for the work queued on
+    the current stream (its inputs, and outputs this module just zeroed there)."""
+    if stream is not None:
+        stream.wait_stream(torch.cuda.current_stream(stream.device))
+
+
+def _leave(stream) -> None:
+    """... and the current stream waits for the call before its result is used
+    (or freed) there."""
+    if stream is not None:
+        torch.cuda.current_stream(stream.device).wait_stream(stream)
+
+
 def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
@@ -220,9 +234,11 @@ def chunk_reduce(x: torch.Tensor, problem: Problem, stream=None) -> torch.Tensor
     _require(x, "x")
     T, H, d = x.shape
     out = torch.empty(H, problem.num_chunks, d, dtype=torch.float32, device=x.device)
+    _enter(stream)
     _check(lib().dhsa_chunk_reduce(_ptr(x), _dtype_code(x), T, H, d, _ptr(problem.d_bounds),
                                    problem.num_chunks, _ptr(out), _stream_ptr(stream)),
            "dhsa_chunk_reduce")
+    _leave(stream)
     return out
 
 
@@ -230,8 +246,10 @@ def chunk_similarity(qc: torch.Tensor, kc: torch.Tensor, problem: Problem, strea
     """Step 2: fp32 [Hq, n, n]; entries outside the causal same-sequence triangle are 0."""
     n = problem.num_chunks
     scores = torch.zeros(problem.num_q_heads, n, n, dtype=torch.float32, device=qc.device)
+    _enter(stream)
     _check(lib().dhsa_chunk_similarity(_ptr(qc), _ptr(kc), problem.ref(), _ptr(scores),
                                        _stream_ptr(stream)), "dhsa_chunk_similarity")
+    _leave(stream)
     return scores
 
 
@@ -245,15 +263,19 @@ def topk_select(scores: torch.Tensor, problem: Problem, budget: Budget, stream=N
     col = torch.empty(max(nnz, 1), dtype=torch.int32, device=dev)
     ws = _workspace(256, dev)
     st = _stream_ptr(stream)
+    _enter(stream)
     _check(lib().dhsa_topk_select(_ptr(scores), problem.ref(), _budget(budget), _ptr(row_ptr), _ptr(col),
                                   nnz, _ptr(ws), ws.numel(), st), "dhsa_topk_select")
     if check:
         _check(lib().dhsa_workspace_status(_ptr(ws), st), "dhsa_topk_select (device)")
+    _leave(stream)
     return Plan(row_ptr, col[:nnz], nnz, bool(budget.per_kv_head))
 
 
 class Planner:
-    """Owns the plan workspace and output buffers for repeated dhsa_plan calls."""
+    """Owns the plan workspace and output buffers for repeated dhsa_plan calls.
+    With an explicit stream, ordering against other streams is the caller's
+    (the one-shot functions below do it themselves)."""
 
     def __init__(self, problem: Problem, budget: Budget, device=None):
         self.problem, self.budget = problem, budget
@@ -281,14 +303,17 @@ def plan(q: torch.Tensor, k: torch.Tensor, problem: Problem, budget: Budget, str
     _require(q, "q")
     _require(k, "k")
     p = Planner(problem, budget, q.device)
+    _enter(stream)
     out = p(q, k, stream)
     if check:
         _check(p.status(stream), "dhsa_plan (device)")
+    _leave(stream)
     return Plan(out.row_ptr.clone(), out.col.clone(), out.nnz, out.per_kv_head)
 
 
 class Attention:
-    """Owns the attention workspace for repeated dhsa_attention calls."""
+    """Owns the attention workspace for repeated dhsa_attention calls (stream
+    ordering as for Planner)."""
 
     def __init__(self, problem: Problem, device=None):
         self.problem = problem
@@ -314,9 +339,11 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, problem: Proble
         _require(t, name)
     out = torch.empty_like(q)
     a = Attention(problem, q.device)
+    _enter(stream)
     a(q, k, v, plan, out, scale, stream)
     if check:
         _check(a.status(stream), "dhsa_attention (device)")
+    _leave(stream)
     return out
 
 
@@ -365,9 +392,11 @@ def segment(k: torch.Tensor, cu_seqlens, rule, stream=None, check: bool = False)
     Waits for the result and returns host int32 arrays (chunk_bounds [n+1],
     seq_chunk_ptr [B+1]), ready for ``Problem``."""
     seg = Segmenter(cu_seqlens, k.shape[1], k.shape[2], rule, k.device)
+    _enter(stream)
     bounds, ptr, n = seg(k, stream)
     if check:
         _check(seg.status(stream), "dhsa_segment (device)")
+    _leave(stream)
     n = int(n.item())
     return bounds[:n + 1].cpu().numpy(), ptr.cpu().numpy()
 

@@ -312,6 +312,33 @@ def test_concurrent_calls_on_two_streams():
             assert torch.equal(out, ref), rep
 
 
+def test_one_shot_calls_on_a_side_stream():
+    """The one-shot functions given a side stream order themselves against the
+    current stream (inputs, zeroed outputs, and the result's use there) and give
+    the same results as on the current stream."""
+    inp = _case("d128_long_runs")
+    q, k, v, prob = to_device(inp)
+    ref_plan = api.plan(q, k, prob, inp.budget, check=True)
+    ref_out = api.attention(q, k, v, prob, ref_plan, check=True)
+    ref_qc = api.chunk_reduce(q, prob)
+    ref_kc = api.chunk_reduce(k, prob)
+    ref_s = api.chunk_similarity(ref_qc, ref_kc, prob)
+    torch.cuda.synchronize()
+    st = torch.cuda.Stream()
+    for rep in range(2):
+        plan = api.plan(q, k, prob, inp.budget, stream=st, check=True)
+        out = api.attention(q, k, v, prob, plan, stream=st, check=True)
+        qc = api.chunk_reduce(q, prob, stream=st)
+        kc = api.chunk_reduce(k, prob, stream=st)
+        sc = api.chunk_similarity(qc, kc, prob, stream=st)
+        sel = api.topk_select(sc, prob, inp.budget, stream=st, check=True)
+        # used on the current stream without any explicit synchronisation
+        assert torch.equal(plan.row_ptr, ref_plan.row_ptr) and torch.equal(plan.col, ref_plan.col), rep
+        assert torch.equal(sel.row_ptr, ref_plan.row_ptr) and torch.equal(sel.col, ref_plan.col), rep
+        assert torch.equal(out, ref_out), rep
+        assert torch.equal(qc, ref_qc) and torch.equal(kc, ref_kc) and torch.equal(sc, ref_s), rep
+
+
 def test_empty_sequence_in_batch():
     inp = W.random_problem(7, [500, 0, 300], 2, 1, 64, "bf16", 40, 120, W.Budget.topk(2))
     q, k, v, prob = to_device(inp)
