@@ -381,7 +381,8 @@ def bench_gpu(args):
                 "schedule": "each step copies Q/K/V in from pinned host memory and O out; copy-in, "
                             "plan + attention and copy-out of consecutive steps overlap on three streams "
                             "(three device buffer sets)"},
-        "gpu_launches": 4 * args.steps,
+        # per step: chunk reduce (Q and K in one launch), [group sum,] similarity, select, attention
+        "gpu_launches": (5 if args.kv_plan else 4) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -455,6 +456,7 @@ def bench_select_micro(args):
         "roofline": {"kernel": "topk_select_kernel", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "peak_kind": "%s copy bandwidth" % peaks["source"]},
+        "gpu_launches": args.steps,  # one select kernel per call
     }), flush=True)
 
 
@@ -516,6 +518,7 @@ def bench_segment_micro(args):
                      "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "peak_kind": "%s copy bandwidth" % peaks["source"],
                      "note": "whole call timed: the walk and compaction count against it"},
+        "gpu_launches": 3 * args.steps,  # similarity, walk, compaction per call
         "clocks": clk,
     }
     if not args.no_cpu_baseline:
@@ -596,6 +599,7 @@ def bench_online_chunking(args):
                    "rule": {"threshold": rule.threshold, "min_len": rule.min_len, "max_len": rule.max_len},
                    "num_chunks": int(hb.shape[0] - 1), "budget": _budget_str(inp.budget)},
         "ms_segment_and_readback": part[0], "ms_plan": part[1], "ms_attention": part[2],
+        "gpu_launches": 7 * args.steps,  # segment 3, plan 3, attention 1 per step
         "clocks": clk,
     }), flush=True)
 
