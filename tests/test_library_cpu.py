@@ -41,6 +41,20 @@ def test_library_exports_every_declared_symbol():
     assert exported == _declared_symbols()
 
 
+def test_binding_signatures_match_the_header():
+    """Every entry point takes as many arguments in the binding as the header
+    declares (a dropped or extra argument would shift every later one)."""
+    hdr = open(os.path.join(ROOT, "include", "dhsa.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    hdr = re.sub(r"//[^\n]*", "", hdr)
+    L = api.lib()
+    for name in api.EXPORTED:
+        m = re.search(r"\b%s\s*\(([^;{]*)\)\s*;" % name, hdr, re.S)
+        assert m, name
+        params = [q for q in m.group(1).split(",") if q.strip() and q.strip() != "void"]
+        assert len(params) == len(getattr(L, name).argtypes), name
+
+
 def test_status_strings():
     L = api.lib()
     for code, name in api.STATUS_NAMES.items():
