@@ -34,7 +34,7 @@ EXPORTED = [
     "dhsa_chunk_similarity", "dhsa_topk_select", "dhsa_plan_workspace_size", "dhsa_plan",
     "dhsa_attention_workspace_size", "dhsa_attention", "dhsa_workspace_status",
     "dhsa_selftest_timeout", "dhsa_plan_noalloc", "dhsa_attention_kv_plan",
-    "dhsa_segment_capacity", "dhsa_segment_workspace_size", "dhsa_segment",
+    "dhsa_segment_capacity", "dhsa_segment_workspace_size", "dhsa_segment", "dhsa_plan_check",
 ]
 
 DHSA_BUDGET_PER_KV_HEAD = 0x100
@@ -103,6 +103,7 @@ def lib() -> ctypes.CDLL:
             "dhsa_segment_capacity": (ctypes.c_int, [P, I32, I32, ctypes.POINTER(I64)]),
             "dhsa_segment_workspace_size": (ctypes.c_int, [I32, ctypes.POINTER(SZ)]),
             "dhsa_segment": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, _SegmentRule, P, I64, P, P, P, SZ, P]),
+            "dhsa_plan_check": (ctypes.c_int, [PP, P, P, I64, I32, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -309,6 +310,25 @@ def plan(q: torch.Tensor, k: torch.Tensor, problem: Problem, budget: Budget, str
         _check(p.status(stream), "dhsa_plan (device)")
     _leave(stream)
     return Plan(out.row_ptr.clone(), out.col.clone(), out.nnz, out.per_kv_head)
+
+
+def check_plan(problem: Problem, row_ptr: torch.Tensor, col: torch.Tensor, per_kv_head: bool = False,
+               stream=None) -> int:
+    """Device-side structural check of a plan (dhsa_plan_check).  Waits for it
+    and returns the status (0 = a valid plan, 6 = DHSA_ERR_DEVICE_CHECK).
+    row_ptr / col: int32 device tensors; nnz = col.numel()."""
+    _require(row_ptr, "row_ptr")
+    _require(col, "col")
+    if row_ptr.dtype != torch.int32 or col.dtype != torch.int32:
+        raise TypeError("row_ptr and col must be int32")
+    ws = _workspace(256, row_ptr.device)
+    st = _stream_ptr(stream)
+    _enter(stream)
+    _check(lib().dhsa_plan_check(problem.ref(), _ptr(row_ptr), _ptr(col), int(col.numel()), int(bool(per_kv_head)),
+                                 _ptr(ws), ws.numel(), st), "dhsa_plan_check")
+    code = int(lib().dhsa_workspace_status(_ptr(ws), st))
+    _leave(stream)
+    return code
 
 
 class Attention:

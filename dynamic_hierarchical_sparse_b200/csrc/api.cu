@@ -150,7 +150,7 @@ dhsa_status run_plan(const void* q, const void* k, const dhsa_problem* p, const 
 dhsa_status run_attention(const void* q, const void* k, const void* v, const dhsa_problem* p,
                           const int32_t* row_ptr, const int32_t* col, int64_t nnz, int plan_group, float scale,
                           void* out, void* workspace, size_t workspace_bytes, cudaStream_t st) {
-  if (nnz < static_cast<int64_t>(p->num_q_heads / plan_group) * p->num_chunks)
+  if (nnz < static_cast<int64_t>(p->num_q_heads / plan_group) * p->num_chunks || nnz > INT32_MAX)
     return DHSA_ERR_INVALID_ARG;  // >= diagonal per row
   if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
   if (p->total_tokens == 0 || p->num_chunks == 0) return DHSA_OK;
@@ -164,8 +164,9 @@ dhsa_status run_attention(const void* q, const void* k, const void* v, const dhs
   if (p->dtype == DHSA_F32) {
     return cuda_status(launch_attention_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                             static_cast<const float*>(v), p->chunk_bounds, p->num_chunks, row_ptr,
-                                            col, p->total_tokens, p->num_q_heads, p->num_kv_heads, p->head_dim,
-                                            plan_group, scale, static_cast<float*>(out), st));
+                                            col, static_cast<int>(nnz), p->total_tokens, p->num_q_heads,
+                                            p->num_kv_heads, p->head_dim, plan_group, scale,
+                                            static_cast<float*>(out), status, st));
   }
   AttnBf16Args a;
   a.q = q;
@@ -175,6 +176,7 @@ dhsa_status run_attention(const void* q, const void* k, const void* v, const dhs
   a.bounds = p->chunk_bounds;
   a.row_ptr = row_ptr;
   a.col = col;
+  a.nnz = static_cast<int>(nnz);
   a.num_chunks = p->num_chunks;
   a.total_tokens = p->total_tokens;
   a.num_q_heads = p->num_q_heads;
@@ -359,6 +361,22 @@ dhsa_status dhsa_attention_kv_plan(const void* q, const void* k, const void* v, 
   if (s != DHSA_OK) return s;
   return run_attention(q, k, v, p, row_ptr, col, nnz, p->num_q_heads / p->num_kv_heads, scale, out, workspace,
                        workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+dhsa_status dhsa_plan_check(const dhsa_problem* p, const int32_t* row_ptr, const int32_t* col, int64_t nnz,
+                            int32_t per_kv_head, void* workspace, size_t workspace_bytes, void* stream) {
+  dhsa_status s = check_problem(p);
+  if (s != DHSA_OK) return s;
+  const int64_t rows = static_cast<int64_t>(per_kv_head ? p->num_kv_heads : p->num_q_heads) * p->num_chunks;
+  if (nnz < rows || nnz > INT32_MAX) return DHSA_ERR_INVALID_ARG;  // every row holds at least its diagonal
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
+  if (rows == 0) return DHSA_OK;
+  if (row_ptr == nullptr || col == nullptr) return DHSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DHSA_ERR_CUDA;
+  return cuda_status(launch_plan_check(row_ptr, col, nnz, static_cast<int>(rows), p->num_chunks, p->seq_chunk_ptr,
+                                       p->num_seqs, status, st));
 }
 
 dhsa_status dhsa_workspace_status(const void* workspace, void* stream) {

@@ -76,12 +76,14 @@ enum {
 // Walks the key tiles of one work item: runs of consecutive kept chunks, cut
 // into BN-token tiles; every run is clipped at `cap` (one past the tile's last
 // valid query row), which only ever shortens the run holding the diagonal.
+// Plan entries outside [0, num_chunks) are clamped into it (so the bounds are
+// never read out of range) and counted in `bad`, which the caller reports.
 template <int BN>
 struct KeyTiles {
   const int* col;
   const int* bounds;
-  int p, pend, re, k0, cap;
-  __device__ void init(const int* col_, const int* bounds_, int p0, int p1, int cap_) {
+  int p, pend, re, k0, cap, nch, bad;
+  __device__ void init(const int* col_, const int* bounds_, int p0, int p1, int cap_, int num_chunks) {
     col = col_;
     bounds = bounds_;
     p = p0;
@@ -89,17 +91,27 @@ struct KeyTiles {
     re = 0;
     k0 = 0;
     cap = cap_;
+    nch = num_chunks;
+    bad = 0;
+  }
+  __device__ int chunk(int q) {
+    const int c = col[q];
+    if (static_cast<unsigned>(c) >= static_cast<unsigned>(nch)) {
+      ++bad;
+      return min(max(c, 0), nch - 1);
+    }
+    return c;
   }
   __device__ bool next(int& tile_k0, int& tile_end) {
     if (k0 + BN < re) {
       k0 += BN;
     } else {
       if (p >= pend) return false;
-      int c = col[p++];
+      int c = chunk(p++);
       const int rs = bounds[c];
       int e = bounds[c + 1];
-      while (p < pend && col[p] == c + 1) {
-        c = col[p++];
+      while (p < pend && chunk(p) == c + 1) {
+        c = chunk(p++);
         e = bounds[c + 1];
       }
       re = min(e, cap);
@@ -121,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attention_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                           const int* __restrict__ bounds, const int* __restrict__ row_ptr,
-                          const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
+                          const int* __restrict__ col, int nnz, int num_chunks, int num_q_heads, int group,
                           int plan_group, float scale_log2, uint32_t* status) {
   using C = Cfg<D, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -143,7 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q_end = min(q0 + kBM, c_end);
   const int g = h / group;
   const int r = (h / plan_group) * num_chunks + ci;
-  const int p0 = row_ptr[r], p1 = row_ptr[r + 1];
+  int p0 = row_ptr[r], p1 = row_ptr[r + 1];
+  const bool bad_row = p0 < 0 || p1 < p0 || p1 > nnz;
+  if (bad_row) p0 = p1 = 0;  // a malformed plan row is reported below and walked as an empty row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -176,9 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int ntiles = 0;
   {
     KeyTiles<BN> it;
-    it.init(col, bounds, p0, p1, q_end);
+    it.init(col, bounds, p0, p1, q_end, num_chunks);
     int a, b;
     while (it.next(a, b)) ++ntiles;
+    if (threadIdx.x == 0 && (bad_row || it.bad)) report(status, kDevCheck);
   }
 
   if (warp == kProducerWarp) {
@@ -191,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int a = 0; a < D / 64; ++a)
         tma_load_3d(sbase + C::kOffQ + a * C::kQSub, &tm_q, bar(kBarQ), a * 64, h, q0);
       KeyTiles<BN> it;
-      it.init(col, bounds, p0, p1, q_end);
+      it.init(col, bounds, p0, p1, q_end, num_chunks);
       int k0, ke;
       int issued = 0;
       for (int t = 0; it.next(k0, ke); ++t) {
@@ -277,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY;  // running max of logits * scale * log2(e)
     float l_run = 0.f;
     KeyTiles<BN> it;
-    it.init(col, bounds, p0, p1, q_end);
+    it.init(col, bounds, p0, p1, q_end, num_chunks);
     int k0, ke;
     bool ok = true;
     for (int j = 0; it.next(k0, ke); ++j) {
@@ -441,7 +456,7 @@ cudaError_t launch_dim(const AttnBf16Args& a, cudaStream_t stream) {
   dim3 grid(mtiles, a.num_q_heads, a.num_chunks);
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
-                                                  a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
+                                                  a.row_ptr, a.col, a.nnz, a.num_chunks, a.num_q_heads,
                                                   a.num_q_heads / a.num_kv_heads, a.plan_group, scale_log2,
                                                   a.status);
   return cudaGetLastError();

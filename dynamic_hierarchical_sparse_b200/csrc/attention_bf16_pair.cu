@@ -60,7 +60,6 @@
 // (only when a warp's running max grows by more than 2^8; two rounds of two
 // 32-column TMEM slices with packed multiplies).
 #include "common.cuh"
-#include "exp2_poly.cuh"
 #include "launchers.h"
 
 namespace dhsa {
@@ -71,12 +70,6 @@ constexpr int kBN = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t kRegsSoftmax = 224;  // 8 warps x 224 + 4 warps x 56 = 384 x 168
 constexpr uint32_t kRegsOther = 56;
-// Every kPolyPairEvery-th pair of softmax columns takes its exp2 on the FMA
-// pipe (exp2_fma) instead of the MUFU unit; 0 keeps every exp2 on MUFU.
-constexpr int kPolyPairEvery = 0;
-// Two exponentials per MUFU operation (ex2.approx.f16x2): the arguments are
-// rounded to fp16 (11-bit significand), finer than the bf16 the results feed.
-constexpr bool kExpHalf2 = false;
 // P is handed to the tensor core in two halves of 64 keys: the PV product of
 // the first half runs while the softmax exponentiates the second.
 constexpr bool kSplitP = true;
@@ -145,6 +138,18 @@ struct Item {
 };
 static_assert(sizeof(Item) == 64, "item slot size");
 
+// A plan entry read from the caller's plan, clamped into [0, num_chunks) so
+// that a malformed plan never indexes the chunk bounds out of range (the
+// scheduler reports such an entry; every role clamps it the same way).
+__device__ __forceinline__ int plan_chunk(const int* __restrict__ col, int p, int num_chunks) {
+  const int c = col[p];
+  return min(max(c, 0), num_chunks - 1);
+}
+
+__device__ __forceinline__ bool chunk_in_range(int c, int num_chunks) {
+  return static_cast<unsigned>(c) < static_cast<unsigned>(num_chunks);
+}
+
 // Key tiles of one work item: cached runs first, then (if the run list
 // overflowed) runs merged on the fly from the plan in global memory.
 struct TileWalk {
@@ -152,10 +157,10 @@ struct TileWalk {
   int ncached, r;
   const int* col;
   const int* bounds;
-  int p, pend;
+  int p, pend, nch;
   int k0, re, cap;
   __device__ __forceinline__ void init(const int2* ranges_, int ncached_, const int* col_, const int* bounds_, int resume,
-                       int p1, int cap_) {
+                       int p1, int cap_, int num_chunks) {
     ranges = ranges_;
     ncached = ncached_;
     r = 0;
@@ -163,6 +168,7 @@ struct TileWalk {
     bounds = bounds_;
     p = resume;
     pend = p1;
+    nch = num_chunks;
     k0 = 0;
     re = 0;
     cap = cap_;
@@ -176,11 +182,11 @@ struct TileWalk {
       re = min(g.y, cap);
     } else {
       if (p >= pend) return false;
-      int c = col[p++];
+      int c = plan_chunk(col, p++, nch);
       const int rs = bounds[c];
       int e = bounds[c + 1];
-      while (p < pend && col[p] == c + 1) {
-        c = col[p++];
+      while (p < pend && plan_chunk(col, p, nch) == c + 1) {
+        c = plan_chunk(col, p++, nch);
         e = bounds[c + 1];
       }
       k0 = rs;
@@ -200,24 +206,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// exp2 of two fp32 arguments through one ex2.approx.f16x2; results widened to fp32.
-__device__ __forceinline__ float2 ex2_pair_f16(float x0, float x1) {
-  uint32_t h;
-  asm("{\n\t.reg .b32 t;\n\t"
-      "cvt.rn.f16x2.f32 t, %2, %1;\n\t"
-      "ex2.approx.f16x2 %0, t;\n\t}"
-      : "=r"(h)
-      : "f"(x0), "f"(x1));
-  float2 r;
-  asm("{\n\t.reg .b16 lo, hi;\n\t"
-      "mov.b32 {lo, hi}, %2;\n\t"
-      "cvt.f32.f16 %0, lo;\n\t"
-      "cvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "r"(h));
   return r;
 }
 
@@ -272,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attention_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                           const int* __restrict__ bounds, const int* __restrict__ row_ptr,
-                          const int* __restrict__ col, int num_chunks, int num_q_heads, int group,
+                          const int* __restrict__ col, int nnz, int num_chunks, int num_q_heads, int group,
                           int plan_group, int head_pair, int tiles, int total_items, float scale_log2,
                           uint32_t* status, int* item_counter) {
   using C = PairCfg<D>;
@@ -368,7 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q_end1 = valid1 ? min(q01 + kBM, c_end) : q01;
         const int cap = valid1 ? q_end1 : q_end0;
         const int row_id = (hh / plan_group) * num_chunks + ci;
-        const int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
+        int p0 = row_ptr[row_id], p1 = row_ptr[row_id + 1];
+        if (p0 < 0 || p1 < p0 || p1 > nnz) {
+          // a malformed plan row: reported, and walked as an empty row
+          if (lane == 0) report(status, kDevCheck);
+          p0 = p1 = 0;
+        }
         // merge the row's kept chunks into runs of consecutive chunks
         if (lane == 0) d->resume = p1;
         __syncwarp();
@@ -376,11 +369,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int base = p0; base < p1; base += 32) {
           const int p = base + lane;
           const bool valid = p < p1;
-          const int c = valid ? col[p] : 0;
+          const int c = valid ? plan_chunk(col, p, num_chunks) : 0;
+          if (valid && !chunk_in_range(col[p], num_chunks)) report(status, kDevCheck);
           int cprev = __shfl_up_sync(0xffffffffu, c, 1);
           int cnext = __shfl_down_sync(0xffffffffu, c, 1);
-          if (lane == 0) cprev = (p > p0) ? col[p - 1] : -2;
-          if (lane == 31) cnext = (p + 1 < p1) ? col[p + 1] : -2;
+          if (lane == 0) cprev = (p > p0) ? plan_chunk(col, p - 1, num_chunks) : -2;
+          if (lane == 31) cnext = (p + 1 < p1) ? plan_chunk(col, p + 1, num_chunks) : -2;
           const bool is_start = valid && (p == p0 || c != cprev + 1);
           const bool is_end = valid && (p == p1 - 1 || cnext != c + 1);
           const unsigned sm = __ballot_sync(0xffffffffu, is_start);
@@ -403,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // key tiles of the item (tile 1, or the only tile) and tile 0's prefix
           int nt = 0, nt0 = 0;
           TileWalk w;
-          w.init(ranges, ncached, col, bounds, d->resume, p1, cap);
+          w.init(ranges, ncached, col, bounds, d->resume, p1, cap, num_chunks);
           int k0, ke;
           while (w.next(k0, ke)) {
             ++nt;
@@ -456,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         qloads = k + 1;
         const int g = d.h / group;
         TileWalk w;
-        w.init(ranges_all + s * kRangeCap, d.ncached, col, bounds, d.resume, d.p1, d.cap);
+        w.init(ranges_all + s * kRangeCap, d.ncached, col, bounds, d.resume, d.p1, d.cap, num_chunks);
         int k0, ke;
         for (int t = 0; w.next(k0, ke); ++t) {
           const int tg = T + t;  // key tile counted across items
@@ -622,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY;  // running max of logits * scale * log2(e)
     float l_run = 0.f;
     TileWalk w;
-    w.init(ranges_all + slot * kRangeCap, d.ncached, col, bounds, d.resume, d.p1, d.cap);
+    w.init(ranges_all + slot * kRangeCap, d.ncached, col, bounds, d.resume, d.p1, d.cap, num_chunks);
     int k0, ke;
     for (int t = 0; t < nta && w.next(k0, ke); ++t) {
       if (!mbar_wait(bar(kBarSFull + a), ns & 1, abort_flag, status)) {
@@ -701,18 +695,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             x0 = fmaf(s[c], scale_log2, -m_use);
             x1 = fmaf(s[c + 1], scale_log2, -m_use);
           }
-          float e0, e1;
-          if (kExpHalf2) {
-            const float2 e = ex2_pair_f16(x0, x1);
-            e0 = e.x;
-            e1 = e.y;
-          } else if (kPolyPairEvery > 0 && (c / 2) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
-            e0 = exp2_fma(x0);
-            e1 = exp2_fma(x1);
-          } else {
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          }
+          const float e0 = ex2_approx(x0);
+          const float e1 = ex2_approx(x1);
           if (kPackedF32)
             ps2[(c / 2) & 1] = f2_add(ps2[(c / 2) & 1], f2_pack(e0, e1));
           else
@@ -846,7 +830,7 @@ cudaError_t launch_attention_pair_dim(const AttnBf16Args& a, cudaStream_t stream
   const int grid = static_cast<int>(total < sms ? total : sms);
   const float scale_log2 = a.scale * 1.4426950408889634f;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(a.out), a.bounds,
-                                                  a.row_ptr, a.col, a.num_chunks, a.num_q_heads,
+                                                  a.row_ptr, a.col, a.nnz, a.num_chunks, a.num_q_heads,
                                                   a.num_q_heads / a.num_kv_heads, a.plan_group, head_pair, tiles,
                                                   static_cast<int>(total), scale_log2, a.status,
                                                   reinterpret_cast<int*>(a.status + 1));

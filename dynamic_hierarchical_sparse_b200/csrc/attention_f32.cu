@@ -24,9 +24,9 @@ template <int D>
 __global__ void __launch_bounds__(kRowsPerCta * 32)
     attention_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                          const float* __restrict__ v, const int* __restrict__ bounds, int num_chunks,
-                         const int* __restrict__ row_ptr, const int* __restrict__ col, int total_tokens,
+                         const int* __restrict__ row_ptr, const int* __restrict__ col, int nnz, int total_tokens,
                          int num_q_heads, int num_kv_heads, int plan_group, float scale,
-                         float* __restrict__ out) {
+                         float* __restrict__ out, uint32_t* status) {
   constexpr int PER = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kRowsPerCta + warp;
@@ -54,8 +54,19 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
 
   const size_t kv_stride = static_cast<size_t>(num_kv_heads) * D;
   const int r = (h / plan_group) * num_chunks + ci;
-  for (int p = row_ptr[r]; p < row_ptr[r + 1]; ++p) {
-    const int cj = col[p];
+  int p0 = row_ptr[r], p1 = row_ptr[r + 1];
+  if (p0 < 0 || p1 < p0 || p1 > nnz) {
+    // a malformed plan row: reported, and walked as an empty row
+    if (lane == 0) report(status, kDevCheck);
+    p0 = p1 = 0;
+  }
+  for (int p = p0; p < p1; ++p) {
+    int cj = col[p];
+    if (static_cast<unsigned>(cj) >= static_cast<unsigned>(num_chunks)) {
+      // an entry outside the chunk range: reported and skipped
+      if (lane == 0) report(status, kDevCheck);
+      continue;
+    }
     const int s0 = bounds[cj];
     const int s1 = min(bounds[cj + 1], t + 1);  // causal
     for (int sb = s0; sb < s1; sb += 32) {
@@ -100,26 +111,26 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
 }  // namespace
 
 cudaError_t launch_attention_f32(const float* q, const float* k, const float* v, const int* bounds,
-                                 int num_chunks, const int* row_ptr, const int* col, int total_tokens,
+                                 int num_chunks, const int* row_ptr, const int* col, int nnz, int total_tokens,
                                  int num_q_heads, int num_kv_heads, int head_dim, int plan_group, float scale,
-                                 float* out, cudaStream_t stream) {
+                                 float* out, uint32_t* status, cudaStream_t stream) {
   if (total_tokens <= 0) return cudaSuccess;
   dim3 grid((total_tokens + kRowsPerCta - 1) / kRowsPerCta, num_q_heads);
   switch (head_dim) {
     case 64:
       attention_f32_kernel<64><<<grid, kRowsPerCta * 32, 0, stream>>>(
-          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, plan_group, scale,
-          out);
+          q, k, v, bounds, num_chunks, row_ptr, col, nnz, total_tokens, num_q_heads, num_kv_heads, plan_group,
+          scale, out, status);
       break;
     case 128:
       attention_f32_kernel<128><<<grid, kRowsPerCta * 32, 0, stream>>>(
-          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, plan_group, scale,
-          out);
+          q, k, v, bounds, num_chunks, row_ptr, col, nnz, total_tokens, num_q_heads, num_kv_heads, plan_group,
+          scale, out, status);
       break;
     case 256:
       attention_f32_kernel<256><<<grid, kRowsPerCta * 32, 0, stream>>>(
-          q, k, v, bounds, num_chunks, row_ptr, col, total_tokens, num_q_heads, num_kv_heads, plan_group, scale,
-          out);
+          q, k, v, bounds, num_chunks, row_ptr, col, nnz, total_tokens, num_q_heads, num_kv_heads, plan_group,
+          scale, out, status);
       break;
     default:
       return cudaErrorInvalidValue;

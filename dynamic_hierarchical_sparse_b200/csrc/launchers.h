@@ -39,10 +39,12 @@ cudaError_t launch_topk_select(const float* scores, int num_chunks, int num_q_he
 
 // Step 4, fp32.  plan_group: query heads per plan row (1: a plan row per query
 // head; Hq/Hkv: a plan row per KV head, read by every head of the group).
+// Plan rows outside [0, nnz] and entries outside [0, num_chunks) are reported
+// in *status (kDevCheck) and skipped.
 cudaError_t launch_attention_f32(const float* q, const float* k, const float* v, const int* bounds,
-                                 int num_chunks, const int* row_ptr, const int* col, int total_tokens,
+                                 int num_chunks, const int* row_ptr, const int* col, int nnz, int total_tokens,
                                  int num_q_heads, int num_kv_heads, int head_dim, int plan_group, float scale,
-                                 float* out, cudaStream_t stream);
+                                 float* out, uint32_t* status, cudaStream_t stream);
 
 // Step 4, bf16 on tcgen05.  h_bounds is the host mirror of bounds (used to
 // size the grid).
@@ -54,6 +56,7 @@ struct AttnBf16Args {
   const int* bounds;
   const int* row_ptr;
   const int* col;
+  int nnz;  // entries of col; plan rows reaching past it are reported (kDevCheck)
   int num_chunks;
   int total_tokens;
   int num_q_heads;
@@ -76,6 +79,11 @@ cudaError_t launch_segment(const void* k, int dtype, int total_tokens, int num_k
                            const int* cu_seqlens, int num_seqs, float threshold, int min_len, int max_len,
                            int* chunk_bounds, long long capacity, int* seq_chunk_ptr, int* num_chunks,
                            uint32_t* drop, uint32_t* start_bits, uint32_t* status, cudaStream_t stream);
+
+// Structural check of a plan (rows = plan heads x num_chunks): sets kDevCheck
+// in *status on any violation; reads only row_ptr[0..rows] and col[0..nnz).
+cudaError_t launch_plan_check(const int* row_ptr, const int* col, long long nnz, int rows, int num_chunks,
+                              const int* seq_chunk_ptr, int num_seqs, uint32_t* status, cudaStream_t stream);
 
 // Diagnostic: a kernel whose only wait can never be satisfied, bounded by limit_ns.
 cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);

@@ -160,10 +160,12 @@ __device__ __forceinline__ void bitonic64_desc(uint32_t& v0, uint32_t& v1, int l
 // lies in [lo, hi].  The keys then share every bit above the highest bit where
 // lo and hi differ, so the MSB-first radix starts there: each pass takes the
 // (up to) 8 bits below the bits already fixed.  hist[] is zero on entry and is
-// left zero.
+// left zero.  Should fewer than `keep` keys be written (a defect, which the
+// caller reports), the remaining slots get `fill` (the row's diagonal chunk), so
+// the row never holds an index outside the chunk range.
 template <typename GetKey, typename GetCol>
 __device__ __forceinline__ bool warp_select(int n, int keep, uint32_t lo, uint32_t hi, int* hist, GetKey get_key,
-                                            GetCol get_col, int* __restrict__ out, int lane) {
+                                            GetCol get_col, int* __restrict__ out, int fill, int lane) {
   const uint32_t diff = lo ^ hi;
   int top = diff == 0u ? -1 : 31 - __clz(static_cast<int>(diff));  // highest undecided bit
   uint32_t mask = top < 0 ? 0xFFFFFFFFu : ~((2u << top) - 1u);      // bits already decided
@@ -250,6 +252,9 @@ __device__ __forceinline__ bool warp_select(int n, int keep, uint32_t lo, uint32
       written += __popc(selm);
       eq_seen += __popc(eqm);
     }
+  }
+  if (written < keep) {
+    for (int t = written + lane; t < keep; t += 32) out[t] = fill;
   }
   return written == keep;  // more or fewer would be a defect: reported, never written past the row
 }
@@ -359,7 +364,7 @@ __global__ void __launch_bounds__(kSelThreads)
       __syncwarp();
       ok = warp_select(
           n, keep, tau_key, hi, ws.hist, [&](int t) { return ws.key[t]; },
-          [&](int t) { return c0 + static_cast<int>(ws.idx[t]); }, out, lane);
+          [&](int t) { return c0 + static_cast<int>(ws.idx[t]); }, out, i, lane);
       if (!ok && lane == 0) report(status, kDevCheck);
       return;
     }
@@ -389,7 +394,7 @@ __global__ void __launch_bounds__(kSelThreads)
     hi = __reduce_max_sync(0xffffffffu, hi);
     __syncwarp();
     ok = warp_select(
-        m, keep, lo, hi, ws.hist, [&](int t) { return ws.key[t]; }, [&](int t) { return c0 + t; }, out, lane);
+        m, keep, lo, hi, ws.hist, [&](int t) { return ws.key[t]; }, [&](int t) { return c0 + t; }, out, i, lane);
   } else {
     // select from the row in global memory (read through L2 once per pass)
     for (int j = lane; j < m; j += 32) {
@@ -401,7 +406,7 @@ __global__ void __launch_bounds__(kSelThreads)
     hi = __reduce_max_sync(0xffffffffu, hi);
     ok = warp_select(
         m, keep, lo, hi, ws.hist, [&](int t) { return order_key(__ldg(srow + t)); }, [&](int t) { return c0 + t; },
-        out, lane);
+        out, i, lane);
   }
   if (!ok && lane == 0) report(status, kDevCheck);
 }

@@ -198,6 +198,29 @@ DHSA_API dhsa_status dhsa_attention_kv_plan(const void* q, const void* k, const 
                                            const int32_t* col, int64_t nnz, float scale, void* out,
                                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Device-side check of a plan before it is handed to step 4 (for plans that
+ * did not come from dhsa_plan / dhsa_topk_select, or that were stored and
+ * reloaded).  A plan row (plan head, query chunk i) must hold the kept key
+ * chunks of i plus its diagonal: a non-empty, strictly ascending list of
+ * chunks of i's own sequence, none later than i, whose last entry is i (the
+ * causal keep set of step 3: On-Device page, Abstract; Memory-Constrained
+ * page: causally important dependencies are kept).  row_ptr must start at 0,
+ * never decrease and end at nnz.
+ *   row_ptr     device int32 [rows + 1], rows = Hq * n, or Hkv * n when
+ *               per_kv_head is non-zero
+ *   col         device int32 [nnz]
+ *   workspace   device, >= 256 bytes: its status word is cleared, then set to
+ *               DHSA_ERR_DEVICE_CHECK's bit by any violation; read it with
+ *               dhsa_workspace_status.
+ * The kernel reads only row_ptr[0..rows] and col[0..nnz), so a malformed
+ * plan cannot make it read out of range.  Argument errors (nnz < rows, a
+ * NULL pointer) return before the launch.  The attention kernels themselves
+ * clamp plan entries into range and report out-of-range ones, but accept
+ * other malformed rows (unsorted, later chunks) with unspecified output. */
+DHSA_API dhsa_status dhsa_plan_check(const dhsa_problem* p, const int32_t* row_ptr, const int32_t* col,
+                                     int64_t nnz, int32_t per_kv_head, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
 /* Waits for `stream`, then reads the status word that the kernels of the last
  * call given `workspace` may have set.  Returns DHSA_OK, DHSA_ERR_TIMEOUT or
  * DHSA_ERR_DEVICE_CHECK (or DHSA_ERR_CUDA if the wait itself failed). */

@@ -184,6 +184,16 @@ def test_entry_points_reject_before_launch():
     # timeout self-test limits
     assert L.dhsa_selftest_timeout(ws, 0, null) == 1
     assert L.dhsa_selftest_timeout(null, 100, null) == 3
+    # plan check: fewer entries than rows (every row holds its diagonal), a
+    # missing workspace, a missing plan
+    rows = 2 * p.num_chunks
+    assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), rows - 1, 0, ws, 256, null) == 1
+    assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, 0, null, 0, null) == 3
+    assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, 0, ws, 16, null) == 3
+    assert L.dhsa_plan_check(p.ref(), null, ctypes.c_void_p(16), nnz, 0, ws, 256, null) == 1
+    # per-KV-head rows (Hkv * n) accept fewer entries than per-query-head ones
+    assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), p.num_chunks - 1, 1, ws, 256,
+                             null) == 1
 
 
 def test_empty_problem_is_a_no_op():
@@ -289,6 +299,38 @@ def test_gate_rounding_allowance_is_half_a_bf16_ulp():
     assert np.all(np.abs(r - x) <= half_ulp_bf16(x))
     assert np.abs(r - x).max() > 0.5 * half_ulp_bf16(x[np.argmax(np.abs(r - x))])
     assert half_ulp_bf16(8.0) == 2.0 ** -5 and half_ulp_bf16(7.99) == 2.0 ** -6
+
+
+def test_bf16_gate_is_flat_below_the_rounding_floor():
+    """The bf16 max-abs gate is the flat 2e-2 wherever |O_ref| < 8 (there the
+    exactly rounded output is within 2^-6 < 2e-2 of the reference), and adds
+    half a bf16 ulp only from |O_ref| = 8 up, where that half ulp (2^-5) alone
+    exceeds 2e-2."""
+    from tests.helpers import ATOL_BF16, gate_tolerance, half_ulp_bf16
+    want = np.array([0.0, -0.02, 0.5, 3.99, -4.0, 7.999, -8.0, 8.25, 15.9, 16.0, -100.0])
+    tol = gate_tolerance(want, torch.bfloat16)
+    below = np.abs(want) < 8
+    assert np.all(tol[below] == ATOL_BF16)
+    assert np.all(tol[~below] == ATOL_BF16 + half_ulp_bf16(want[~below]))
+    assert np.all(half_ulp_bf16(want[below]) < ATOL_BF16)
+    assert np.all(half_ulp_bf16(want[~below]) > ATOL_BF16)
+    assert np.all(gate_tolerance(want, torch.float32) == 1e-4)
+
+
+def test_attention_gate_rejects_a_relative_error_the_absolute_gate_misses():
+    """On diffuse outputs (|O| ~ 0.01) a 50 % error stays under the 2e-2
+    absolute gate; the relative Frobenius gate rejects it, and passes the
+    output's own bf16 rounding."""
+    from tests.helpers import attention_gate
+    rng = np.random.default_rng(1)
+    want = 0.008 * rng.standard_normal((512, 128))
+    rounded = torch.from_numpy(want).to(torch.bfloat16)
+    stats = attention_gate(rounded, want, torch.bfloat16)
+    assert stats[3] < 3e-3
+    wrong = torch.from_numpy(want * 1.5)
+    assert np.abs(want * 0.5).max() < 2e-2
+    with pytest.raises(AssertionError, match="relative Frobenius"):
+        attention_gate(wrong, want, torch.bfloat16)
 
 
 def test_segment_capacity_and_workspace():

@@ -30,7 +30,8 @@ def _gpu():
 
 def _noalloc(q, k, prob, budget, nnz):
     dev = q.device
-    row_ptr = torch.full((prob.num_q_heads * prob.num_chunks + 1,), -1, dtype=torch.int32, device=dev)
+    heads = prob.num_kv_heads if budget.per_kv_head else prob.num_q_heads
+    row_ptr = torch.full((heads * prob.num_chunks + 1,), -1, dtype=torch.int32, device=dev)
     col = torch.full((max(nnz, 1),), -1, dtype=torch.int32, device=dev)
     rc = api.lib().dhsa_plan_noalloc(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), prob.ref(),
                                      api._budget(budget), ctypes.c_void_p(row_ptr.data_ptr()),
@@ -60,6 +61,30 @@ def test_noalloc_matches_workspace_plan_on_consecutive_calls():
             torch.cuda.synchronize()
             assert torch.equal(row_ptr, want.row_ptr), (rep, inp.spec.dtype)
             assert torch.equal(col, want.col), (rep, inp.spec.dtype)
+
+
+def test_noalloc_per_kv_head_plan_on_consecutive_calls():
+    """The per-KV-head layout of the fixed scratch (it adds the summed query
+    chunks and moves the score matrix) gives dhsa_plan's per-KV-head plan, bit
+    for bit, on consecutive calls, also after a per-query-head call has left
+    the differently laid out scratch behind."""
+    dev = torch.device("cuda")
+    inp = _case(0)
+    q, k = inp.q.to(dev), inp.k.to(dev)
+    prob = api.Problem.from_inputs(inp, dev)
+    per_q, per_kv = inp.budget, inp.budget.kv()
+    assert prob.plan_workspace_bytes(per_kv) <= MAX_SCRATCH
+    want_kv = api.plan(q, k, prob, per_kv, check=True)
+    want_q = api.plan(q, k, prob, per_q, check=True)
+    assert want_kv.row_ptr.numel() == prob.num_kv_heads * prob.num_chunks + 1
+    for rep in range(2):
+        row_ptr, col = _noalloc(q, k, prob, per_kv, want_kv.nnz)
+        torch.cuda.synchronize()
+        assert torch.equal(row_ptr, want_kv.row_ptr), rep
+        assert torch.equal(col, want_kv.col), rep
+        row_ptr, col = _noalloc(q, k, prob, per_q, want_q.nnz)
+        torch.cuda.synchronize()
+        assert torch.equal(row_ptr, want_q.row_ptr) and torch.equal(col, want_q.col), rep
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
