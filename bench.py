@@ -971,7 +971,7 @@ def bench_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(step_s) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; rank-4 shared component, scale 2)", "impl": "reference",
-        "config": _config(spec, inp, budget, pairs, 1),
+        "config": _config(spec, inp, budget, pairs, int(os.environ.get("WORLD_SIZE", "1"))),
         "step": ("each step is the oracle's full plan plus attention on a seeded sample of (head, query chunk) "
                  "pairs (%.2f%% of kept pairs in the last step); ms_per_step is that sampled step's wall time, "
                  "and value scales its attention time to every kept pair"

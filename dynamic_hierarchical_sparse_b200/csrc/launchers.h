@@ -70,6 +70,8 @@ struct AttnBf16Args {
 cudaError_t launch_attention_bf16(const AttnBf16Args& a, cudaStream_t stream);
 // head_dim 64 / 128: two query tiles per CTA, P kept in TMEM.
 cudaError_t launch_attention_pair(const AttnBf16Args& a, cudaStream_t stream);
+// head_dim 256: one query tile per CTA, 128-key tiles, S double-buffered and P in TMEM.
+cudaError_t launch_attention_d256(const AttnBf16Args& a, cudaStream_t stream);
 // TMA view of a packed THD bf16 tensor (see attention_bf16.cu).
 CUresult encode_qkv_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows);
 
