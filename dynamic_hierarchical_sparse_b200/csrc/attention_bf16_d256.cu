@@ -36,9 +36,9 @@
 //              QK(0), QK(1), PV(0), QK(2), PV(1), ..., PV(nt-1)
 // The tensor core executes one thread's tcgen05 operations in issue order, so
 // QK(j+2), issued after PV(j), overwrites S(j%2) (and P(j) in it) only after
-// PV(j) has read P(j).  The online softmax is fp32 in the exp2 domain with a
-// lazy O rescale (only when a warp's running max grows by more than 2^8), done
-// after PV(j-1) is complete (O-ready barrier) and before P(j) is released.
+// PV(j) has read P(j).  The online softmax is fp32 in the exp2 domain; O is
+// rescaled whenever a warp's running max grows, after PV(j-1) is complete
+// (O-ready barrier) and before P(j) is released.
 #include "common.cuh"
 #include "launchers.h"
 
@@ -52,7 +52,10 @@ constexpr int kThreads = 192;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleLog2 = 8.0f;
+// O is rescaled whenever a warp's running max grows, so the largest weight
+// of a row is exp2(0) = 1, exact in bf16 (a lagging max would leave it rounded,
+// and that rounding would reach O directly).
+constexpr float kRescaleLog2 = 0.0f;
 constexpr int kSlices = kD / 64;        // 64-column slices of a Q / K / V row
 constexpr int kKSlots = 6;              // K ring: 16 KB slices
 constexpr int kSliceBytes = kBN * 128;  // one 64-column slice of a 128-row tile
@@ -431,12 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, shift2), x0, x1);
         const float e0 = ex2_approx(x0);
         const float e1 = ex2_approx(x1);
-        const uint32_t pv = pack_bf16(e0, e1);
-        pk[c / 2] = pv;
-        // the row sum adds the bf16 weights the PV product multiplies, so
-        // O / l is a convex combination of V rows whatever their rounding
-        ps2[(c / 2) & 1] =
-            f2_add(ps2[(c / 2) & 1], f2_pack(__uint_as_float(pv << 16), __uint_as_float(pv & 0xffff0000u)));
+        pk[c / 2] = pack_bf16(e0, e1);
+        ps2[(c / 2) & 1] = f2_add(ps2[(c / 2) & 1], f2_pack(e0, e1));
       }
       // P(j) over the first 64 columns of S(j % 2) (its S values are in registers)
       tmem_st32p(tS + 0, pk);
