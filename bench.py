@@ -45,7 +45,12 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # and it holds only for the kernel source it was captured on: the record
 # keeps the SHA-256 of that source (attention_bf16_pair.cu + common.cuh), and
 # any other source reports traffic as null.
-ATTN_TRAFFIC_CAPTURE = None
+ATTN_TRAFFIC_CAPTURE = {
+    "bytes": 10.48e9,  # 9.44 GB read + 1.04 GB written
+    "source_sha256": "5362b0cea2af71ed7401ddaa5ef1135640c8d70b58ff4dfce32b384d0f4d0746",
+    "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
+                "-k regex:attention_pair -s 1 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-micro"),
+}
 ATTN_KERNEL_SOURCES = ("dynamic_hierarchical_sparse_b200/csrc/attention_bf16_pair.cu",
                        "dynamic_hierarchical_sparse_b200/csrc/common.cuh")
 
