@@ -35,6 +35,7 @@ EXPORTED = [
     "dhsa_attention_workspace_size", "dhsa_attention", "dhsa_workspace_status",
     "dhsa_selftest_timeout", "dhsa_plan_noalloc", "dhsa_attention_kv_plan",
     "dhsa_segment_capacity", "dhsa_segment_workspace_size", "dhsa_segment", "dhsa_plan_check",
+    "dhsa_plan_margins",
 ]
 
 DHSA_BUDGET_PER_KV_HEAD = 0x100
@@ -104,6 +105,7 @@ def lib() -> ctypes.CDLL:
             "dhsa_segment_workspace_size": (ctypes.c_int, [I32, ctypes.POINTER(SZ)]),
             "dhsa_segment": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, _SegmentRule, P, I64, P, P, P, SZ, P]),
             "dhsa_plan_check": (ctypes.c_int, [PP, P, P, I64, I32, P, SZ, P]),
+            "dhsa_plan_margins": (ctypes.c_int, [PP, _Budget, P, P, I64, P, SZ, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -296,6 +298,17 @@ class Planner:
 
     def status(self, stream=None) -> int:
         return lib().dhsa_workspace_status(_ptr(self.ws), _stream_ptr(stream))
+
+    def margins(self, stream=None) -> torch.Tensor:
+        """Selection margins of the plan the last call wrote (dhsa_plan_margins):
+        fp32 [rows, 2], the k-th and (k+1)-th largest admissible scores per row
+        (NaN where there is none)."""
+        rows = self.row_ptr.numel() - 1
+        out = torch.empty(rows, 2, dtype=torch.float32, device=self.row_ptr.device)
+        _check(lib().dhsa_plan_margins(self.problem.ref(), self._b, _ptr(self.row_ptr), _ptr(self.col), self.nnz,
+                                       _ptr(self.ws), self.ws.numel(), _ptr(out), _stream_ptr(stream)),
+               "dhsa_plan_margins")
+        return out
 
 
 def plan(q: torch.Tensor, k: torch.Tensor, problem: Problem, budget: Budget, stream=None,

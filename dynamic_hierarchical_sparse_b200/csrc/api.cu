@@ -363,6 +363,26 @@ dhsa_status dhsa_attention_kv_plan(const void* q, const void* k, const void* v, 
                        workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+dhsa_status dhsa_plan_margins(const dhsa_problem* p, dhsa_budget budget, const int32_t* row_ptr, const int32_t* col,
+                              int64_t nnz, const void* workspace, size_t workspace_bytes, float* margins,
+                              void* stream) {
+  dhsa_status s = dhsa_validate(p, &budget);
+  if (s != DHSA_OK) return s;
+  const int64_t want = nnz_per_head(p, budget) * plan_heads(p, budget);
+  if (nnz != want || want > INT32_MAX) return DHSA_ERR_INVALID_ARG;
+  const PlanLayout L = plan_layout(p, budget);
+  if (workspace == nullptr || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return DHSA_ERR_WORKSPACE;
+  if (p->num_chunks == 0) return DHSA_OK;
+  if (row_ptr == nullptr || col == nullptr || margins == nullptr) return DHSA_ERR_INVALID_ARG;
+  const unsigned char* ws = static_cast<const unsigned char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(const_cast<unsigned char*>(ws));
+  const float* scores = reinterpret_cast<const float*>(ws + L.scores);
+  const int rows = plan_heads(p, budget) * p->num_chunks;
+  return cuda_status(launch_plan_margins(scores, row_ptr, col, nnz, rows, p->num_chunks, p->seq_chunk_ptr,
+                                         p->num_seqs, margins, status, static_cast<cudaStream_t>(stream)));
+}
+
 dhsa_status dhsa_plan_check(const dhsa_problem* p, const int32_t* row_ptr, const int32_t* col, int64_t nnz,
                             int32_t per_kv_head, void* workspace, size_t workspace_bytes, void* stream) {
   dhsa_status s = check_problem(p);

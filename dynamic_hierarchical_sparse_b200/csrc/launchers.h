@@ -87,6 +87,13 @@ cudaError_t launch_segment(const void* k, int dtype, int total_tokens, int num_k
 cudaError_t launch_plan_check(const int* row_ptr, const int* col, long long nnz, int rows, int num_chunks,
                               const int* seq_chunk_ptr, int num_seqs, uint32_t* status, cudaStream_t stream);
 
+// Per plan row r: margins[2r] = smallest kept score (k-th largest admissible),
+// margins[2r + 1] = largest admissible score left out; NaN where there is none.
+// scores: [rows, num_chunks] fp32 (a plan workspace's score matrix).
+cudaError_t launch_plan_margins(const float* scores, const int* row_ptr, const int* col, long long nnz, int rows,
+                                int num_chunks, const int* seq_chunk_ptr, int num_seqs, float* margins,
+                                uint32_t* status, cudaStream_t stream);
+
 // Diagnostic: a kernel whose only wait can never be satisfied, bounded by limit_ns.
 cudaError_t launch_timeout_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -198,6 +198,26 @@ DHSA_API dhsa_status dhsa_attention_kv_plan(const void* q, const void* k, const 
                                            const int32_t* col, int64_t nnz, float scale, void* out,
                                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Selection margins of a plan just written by dhsa_plan (step 3's top-k over
+ * chunk scores: On-Device page, Abstract).  For every plan row r (r = h * n + i,
+ * or g * n + i for a per-KV-head plan):
+ *   margins[2r]     the smallest score among the kept earlier chunks, i.e. the
+ *                   k-th largest admissible score (NaN when the row keeps none);
+ *   margins[2r + 1] the largest admissible score that was left out, i.e. the
+ *                   (k+1)-th (NaN when every admissible chunk is kept).
+ * Rows whose two margins are close (relative to the row's scores) are the
+ * near-tie rows, where rounding in the scores can change the selection.
+ *   p, budget   the problem and budget of the dhsa_plan call
+ *   row_ptr, col, nnz   that call's plan (device)
+ *   workspace   that call's workspace, unchanged since (its score matrix is read)
+ *   margins     device fp32 [rows, 2], written
+ * A plan entry outside its row's candidate range is skipped and reported in the
+ * workspace's status word (DHSA_ERR_DEVICE_CHECK via dhsa_workspace_status).
+ * Argument errors (another nnz, a workspace too small) return before any launch. */
+DHSA_API dhsa_status dhsa_plan_margins(const dhsa_problem* p, dhsa_budget budget, const int32_t* row_ptr,
+                                       const int32_t* col, int64_t nnz, const void* workspace,
+                                       size_t workspace_bytes, float* margins, void* stream);
+
 /* Device-side check of a plan before it is handed to step 4 (for plans that
  * did not come from dhsa_plan / dhsa_topk_select, or that were stored and
  * reloaded).  A plan row (plan head, query chunk i) must hold the kept key

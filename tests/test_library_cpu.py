@@ -191,6 +191,11 @@ def test_entry_points_reject_before_launch():
     assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, 0, null, 0, null) == 3
     assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, 0, ws, 16, null) == 3
     assert L.dhsa_plan_check(p.ref(), null, ctypes.c_void_p(16), nnz, 0, ws, 256, null) == 1
+    # plan margins: another nnz, a workspace smaller than the plan's
+    assert L.dhsa_plan_margins(p.ref(), b, ctypes.c_void_p(16), ctypes.c_void_p(16), nnz + 1, ws, 1 << 30,
+                               ctypes.c_void_p(16), null) == 1
+    assert L.dhsa_plan_margins(p.ref(), b, ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ws, 16,
+                               ctypes.c_void_p(16), null) == 3
     # per-KV-head rows (Hkv * n) accept fewer entries than per-query-head ones
     assert L.dhsa_plan_check(p.ref(), ctypes.c_void_p(16), ctypes.c_void_p(16), p.num_chunks - 1, 1, ws, 256,
                              null) == 1
