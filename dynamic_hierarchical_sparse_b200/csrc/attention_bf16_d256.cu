@@ -23,11 +23,9 @@
 //             so PV is one M=128, N=256 (= d) MMA per 16 keys, the tensor
 //             core's full-rate shape, with no P traffic through shared memory;
 //   O         columns [256, 512).
-// Shared memory: Q (64 KB, four 64-column slices), K streamed as 16 KB slices
-// (128 keys x 64 columns) through a 6-slot ring, each slot released by a
-// commit once the four QK^T MMAs that read it are done (so tile j+1's first
-// slices load while tile j's last ones are still being multiplied), and V as
-// one 64 KB tile released by a commit after its PV.
+// Shared memory: Q (64 KB, four 64-column slices), K as 16 KB slices (128
+// keys x 64 columns) in a 6-slot ring, slice s of key tile t in slot
+// (4t + s) % 6, and V as one 64 KB tile.
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax + epilogue; thread r owns query row r (= TMEM lane r)
@@ -39,6 +37,14 @@
 // PV(j) has read P(j).  The online softmax is fp32 in the exp2 domain; O is
 // rescaled whenever a warp's running max grows, after PV(j-1) is complete
 // (O-ready barrier) and before P(j) is released.
+//
+// The issuing thread runs in step with the tensor pipe, and each barrier test
+// or commit it makes between MMAs leaves the pipe waiting, so the protocol
+// keeps them to three waits (P-full, V-full, K-full) and two commits (O-ready,
+// S-full) per key tile: the four slices of a K tile land on one barrier (one
+// per tile parity), the producer takes the S-full commit of QK(t-1) as the
+// release of the slots that K(t) overwrites (tiles t-2 and t-1), and the
+// O-ready commit of PV(j-1) as the release of V.
 #include "common.cuh"
 #include "launchers.h"
 
@@ -73,11 +79,9 @@ static_assert(2 * kBN + kD <= 512, "TMEM budget");
 
 enum {
   kBarQ = 0,
-  kBarKFull = 1,                    // + slot
-  kBarKEmpty = kBarKFull + kKSlots,  // + slot
-  kBarVFull = kBarKEmpty + kKSlots,
-  kBarVEmpty = kBarVFull + 1,
-  kBarSFull = kBarVEmpty + 1,  // + buffer
+  kBarKFull = 1,              // + (key tile & 1): all four slices of the tile landed
+  kBarVFull = kBarKFull + 2,
+  kBarSFull = kBarVFull + 1,  // + buffer
   kBarPFull = kBarSFull + 2,
   kBarOReady = kBarPFull + 1,
   kBarDrain = kBarOReady + 1,
@@ -223,12 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < kKSlots; ++s) {
-      mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
-    }
+    mbar_init(bar(kBarKFull + 0), 1);
+    mbar_init(bar(kBarKFull + 1), 1);
     mbar_init(bar(kBarVFull), 1);
-    mbar_init(bar(kBarVEmpty), 1);
     mbar_init(bar(kBarSFull + 0), 1);
     mbar_init(bar(kBarSFull + 1), 1);
     mbar_init(bar(kBarPFull), 4);  // one arrival per softmax warp
@@ -269,20 +270,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       KeyTiles kt, vt;
       kt.init(col, bounds, p0, p1, q_end, num_chunks);
       vt.init(col, bounds, p0, p1, q_end, num_chunks);
-      int kslices = 0, vtiles = 0;
+      int ktiles = 0, vtiles = 0, qk_seen = -1;
       bool ok = true;
+      // QK(t) done: the S-full commit of its buffer (the MMAs of one thread
+      // complete in issue order, so it also covers every earlier QK)
+      auto wait_qk = [&](int t) -> bool {
+        if (t <= qk_seen) return true;
+        if (!mbar_wait(bar(kBarSFull + (t & 1)), (t >> 1) & 1, abort_flag, status)) return false;
+        qk_seen = t;
+        return true;
+      };
+      // K(t) as four 16 KB slices, slice u = 4t + s into slot u % kKSlots, all
+      // behind one barrier per tile parity.  The slots' previous slices belong
+      // to tiles t-2 and t-1, free once QK(t-1) is done; waiting for that
+      // before arming means no tile is ever left partly issued.
       auto load_k = [&]() -> bool {
         int k0, ke;
         if (!kt.next(k0, ke)) return true;
-#pragma unroll 1
-        for (int s = 0; s < kSlices; ++s, ++kslices) {
-          const int slot = kslices % kKSlots;
-          if (kslices >= kKSlots &&
-              !mbar_wait(bar(kBarKEmpty + slot), ((kslices / kKSlots) - 1) & 1, abort_flag, status))
-            return false;
-          mbar_arrive_expect_tx(bar(kBarKFull + slot), kSliceBytes);
-          tma_load_3d(sbase + kOffK + slot * kSliceBytes, &tm_k, bar(kBarKFull + slot), s * 64, g, k0);
-        }
+        const int t = ktiles;
+        if (t >= 1 && !wait_qk(t - 1)) return false;
+        mbar_arrive_expect_tx(bar(kBarKFull + (t & 1)), kSlices * kSliceBytes);
+#pragma unroll
+        for (int s = 0; s < kSlices; ++s)
+          tma_load_3d(sbase + kOffK + ((kSlices * t + s) % kKSlots) * kSliceBytes, &tm_k, bar(kBarKFull + (t & 1)),
+                      s * 64, g, k0);
+        ktiles = t + 1;
         return true;
       };
       ok = load_k();
@@ -291,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         int k0, ke;
         vt.next(k0, ke);
-        if (j >= 1 && !mbar_wait(bar(kBarVEmpty), (j - 1) & 1, abort_flag, status)) break;
+        // V(j) replaces V(j-1) once PV(j-1) is done (its O-ready commit)
+        if (j >= 1 && !mbar_wait(bar(kBarOReady), (j - 1) & 1, abort_flag, status)) break;
         mbar_arrive_expect_tx(bar(kBarVFull), kVBytes);
 #pragma unroll
         for (int a = 0; a < kSlices; ++a)
@@ -302,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // let copies already in flight land before the CTA exits (bounded)
         volatile int never = 0;
         mbar_wait(bar(kBarQ), 0, &never, nullptr, 10000000ull);
-        for (int t = max(0, kslices - kKSlots); t < kslices; ++t)
-          mbar_wait(bar(kBarKFull + t % kKSlots), (t / kKSlots) & 1, &never, nullptr, 10000000ull);
+        for (int t = max(0, ktiles - 2); t < ktiles; ++t)
+          mbar_wait(bar(kBarKFull + (t & 1)), (t >> 1) & 1, &never, nullptr, 10000000ull);
         if (vtiles > 0) mbar_wait(bar(kBarVFull), (vtiles - 1) & 1, &never, nullptr, 10000000ull);
       }
     }
@@ -313,16 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, kD, 1);
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, status);
       tc_fence_after();
-      int kslices = 0;
-      // S(j) = Q K(j)^T into buffer j % 2, one K slice (four MMAs) at a time
+      // S(j) = Q K(j)^T into buffer j % 2: one wait for the whole tile
       auto issue_s = [&](int j) -> bool {
         const uint32_t d = tmem + kColS + (j & 1) * kBN;
-#pragma unroll 1
-        for (int s = 0; s < kSlices; ++s, ++kslices) {
-          const int slot = kslices % kKSlots;
-          if (!mbar_wait_spin(bar(kBarKFull + slot), (kslices / kKSlots) & 1, abort_flag, status)) return false;
-          tc_fence_after();
-          const uint32_t kbase = sbase + kOffK + slot * kSliceBytes;
+        if (!mbar_wait_spin(bar(kBarKFull + (j & 1)), (j >> 1) & 1, abort_flag, status)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < kSlices; ++s) {
+          const uint32_t kbase = sbase + kOffK + ((kSlices * j + s) % kKSlots) * kSliceBytes;
           const uint32_t qbase = sbase + kOffQ + s * kSliceBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
@@ -330,9 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = smem_desc_sw128(kbase + kk * 32, 16, 1024);
             umma_f16_ss(d, ad, bd, idesc_s, (s > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(bar(kBarKEmpty + slot));  // the slot is free once these four MMAs are done
         }
-        umma_commit(bar(kBarSFull + (j & 1)));
+        umma_commit(bar(kBarSFull + (j & 1)));  // also frees the tile's K slots
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -347,8 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = smem_desc_sw128(sbase + kOffV + kk * 16 * 128, kSliceBytes, 1024);
           umma_f16_ts(tmem + kColO, pa + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar(kBarVEmpty));
-        umma_commit(bar(kBarOReady));
+        umma_commit(bar(kBarOReady));  // also frees V
         if (j + 2 < ntiles && !issue_s(j + 2)) break;
       }
       // every MMA issued above completes before TMEM is released

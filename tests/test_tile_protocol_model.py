@@ -41,10 +41,15 @@ def test_model_matches_the_kernel_source():
                             "attention_bf16_d256.cu")).read()
     counts = dict(re.findall(r"mbar_init\(bar\((kBar\w+)(?: \+ \w+)?\), (\w+)\)", src))
     assert counts["kBarPFull"] == "4"  # one arrival per softmax warp
-    for name in ("kBarQ", "kBarKFull", "kBarKEmpty", "kBarVFull", "kBarVEmpty", "kBarSFull", "kBarOReady"):
+    for name in ("kBarQ", "kBarKFull", "kBarVFull", "kBarSFull", "kBarOReady"):
         assert counts[name] == "1", name
+    assert "kBarKEmpty" not in src and "kBarVEmpty" not in src
     assert "constexpr int kKSlots = %d;" % TM.K_SLOTS in src
     assert "kSlices = kD / 64" in src and TM.K_SLICES == 256 // 64
+    # slot of slice s of key tile t, and the release the producer waits for
+    assert src.count("((kSlices * t + s) % kKSlots)") == 1 and "((kSlices * j + s) % kKSlots)" in src
+    assert "if (t >= 1 && !wait_qk(t - 1)) return false;" in src
+    assert "!mbar_wait(bar(kBarOReady), (j - 1) & 1, abort_flag, status)) break;" in src
     # the O-ready wait guards every release of P(j), j > 0, not only a rescale
     body = src[src.index("P(j) is released only once PV(j-1) is done"):]
     assert body.index("if (j > 0) {") < body.index("kBarOReady") < body.index("if (any && j > 0)")

@@ -4,13 +4,15 @@ attention kernel for d = 256 (dynamic_hierarchical_sparse_b200/csrc/attention_bf
 One CTA handles one 128-row query tile over `nt` key tiles. Its roles are
 restated as sequential programs, in the kernel's order:
 
-* the TMA producer: Q once; K as 16 KB slices (four per key tile) through a
-  ring of K_SLOTS slots guarded by full/empty barrier pairs, K(j+1) ahead of
-  V(j); V as one tile-sized buffer guarded by its own full/empty pair;
+* the TMA producer: Q once; K as 16 KB slices, slice s of key tile t into
+  ring slot (4t + s) % K_SLOTS, the tile's four slices behind one K-full
+  barrier per tile parity, loaded once QK(t-1) is done (its S-full commit:
+  the slots hold slices of tiles t-2 and t-1); K(j+1) ahead of V(j); V as one
+  tile-sized buffer, reloaded once PV(j-1) is done (its O-ready commit);
 * the single MMA-issuing thread: QK(0), QK(1), then per tile j the PV(j)
-  product (after P-full(j) and V-full(j)) and QK(j+2); each K slice is
-  released by a commit after its four MMAs, S-full(b) after a whole QK^T,
-  V-empty and O-ready after each PV;
+  product (after P-full(j) and V-full(j)) and QK(j+2) (after K-full); it
+  commits S-full(b) after a whole QK^T and O-ready after each PV, nothing
+  else;
 * the four softmax warps: read S(j) from its TMEM buffer j % 2, write P(j)
   over that buffer, wait for O-ready(j-1) (then maybe rescale O), release P(j)
   with one arrival per warp.
@@ -43,9 +45,9 @@ K_SLICES = 4   # 64-column slices of a 256-column K tile
 @dataclasses.dataclass(frozen=True)
 class TileMutation:
     """Protocol slips (each off by default)."""
-    producer_skips_kempty: bool = False   # a K slot refilled without waiting for its MMAs
-    kempty_before_slice: bool = False     # a K slot released before the MMAs that read it
-    producer_skips_vempty: bool = False   # V(j) loaded over V(j-1) without waiting for PV(j-1)
+    producer_skips_qk_wait: bool = False  # K(t) loaded without waiting for QK(t-1)
+    producer_waits_qk_two_back: bool = False  # K(t) loaded after QK(t-2) only (tile t-1's slots)
+    producer_skips_oready: bool = False   # V(j) loaded over V(j-1) without waiting for PV(j-1)
     s_before_pv: bool = False             # QK(j+2) issued before PV(j) (over P(j))
     oready_before_pv: bool = False        # O declared ready (and V free) before PV(j) is issued
     pfull_without_oready: bool = False    # P(j) released without waiting for PV(j-1) unless rescaling
@@ -60,8 +62,8 @@ class TileModel(Model):
         self.rng = rng or random.Random(0)
         self.rescale_prob = rescale_prob
         B = self.bars = {}
-        names = [("Q", 1), ("PFull", 4), ("OReady", 1), ("VFull", 1), ("VEmpty", 1), ("SFull0", 1), ("SFull1", 1)]
-        names += [("KFull%d" % s, 1) for s in range(K_SLOTS)] + [("KEmpty%d" % s, 1) for s in range(K_SLOTS)]
+        names = [("Q", 1), ("PFull", 4), ("OReady", 1), ("VFull", 1), ("SFull0", 1), ("SFull1", 1), ("KFull0", 1),
+                 ("KFull1", 1)]
         for name, count in names:
             B[name] = _Barrier(name, count)
         self.smem = {name: [None, 0] for name in ["Q", "V"] + ["K%d" % s for s in range(K_SLOTS)]}
@@ -78,46 +80,46 @@ class TileModel(Model):
         self.finished = set()
 
     # --------------------------------------------------------------- roles
+    def _kfull(self, t: int):
+        """(barrier, phase) of key tile t's K-full barrier."""
+        return "KFull%d" % (t & 1), t >> 1
+
     def _producer(self):
         nt = self.nt
         yield ("expect", "Q", 0, "prod", 1)
         yield ("tma", "Q", 0, "Q")
-        g = 0
+        seen = [-1]
 
-        def load_k(j):
-            nonlocal g
+        def wait_qk(t):
+            if t < 0 or t <= seen[0]:
+                return
+            yield ("wait", "SFull%d" % (t & 1), t >> 1)
+            seen[0] = t
+
+        def load_k(t):
+            if not self.tmut.producer_skips_qk_wait:
+                yield from wait_qk(t - 2 if self.tmut.producer_waits_qk_two_back else t - 1)
+            bar, n = self._kfull(t)
+            yield ("expect", bar, n, "prod", K_SLICES)
             for s in range(K_SLICES):
-                slot = g % K_SLOTS
-                if g >= K_SLOTS and not self.tmut.producer_skips_kempty:
-                    yield ("wait", "KEmpty%d" % slot, g // K_SLOTS - 1)
-                yield ("expect", "KFull%d" % slot, g // K_SLOTS, "prod", 1)
-                yield ("tma", "K%d" % slot, (j, s), "KFull%d" % slot)
-                g += 1
+                yield ("tma", "K%d" % ((K_SLICES * t + s) % K_SLOTS), (t, s), bar)
 
         yield from load_k(0)
         for j in range(nt):
             if j + 1 < nt:
                 yield from load_k(j + 1)
-            if j >= 1 and not self.tmut.producer_skips_vempty:
-                yield ("wait", "VEmpty", j - 1)
+            if j >= 1 and not self.tmut.producer_skips_oready:
+                yield ("wait", "OReady", j - 1)
             yield ("expect", "VFull", j, "prod", 1)
             yield ("tma", "V", j, "VFull")
 
     def _issuer(self):
         nt = self.nt
-        g = 0
 
         def issue_s(j):
-            nonlocal g
-            for s in range(K_SLICES):
-                slot = g % K_SLOTS
-                yield ("wait", "KFull%d" % slot, g // K_SLOTS)
-                if self.tmut.kempty_before_slice:
-                    yield ("commit", 0, "KEmpty%d" % slot, g // K_SLOTS)
-                yield ("mma", 0, "S", j, s, slot)
-                if not self.tmut.kempty_before_slice:
-                    yield ("commit", 0, "KEmpty%d" % slot, g // K_SLOTS)
-                g += 1
+            bar, n = self._kfull(j)
+            yield ("wait", bar, n)
+            yield ("mma", 0, "S", j)
             yield ("commit", 0, "SFull%d" % (j & 1), j >> 1)
 
         yield ("wait", "Q", 0)
@@ -130,11 +132,9 @@ class TileModel(Model):
             yield ("wait", "PFull", j)
             yield ("wait", "VFull", j)
             if self.tmut.oready_before_pv:
-                yield ("commit", 0, "VEmpty", j)
                 yield ("commit", 0, "OReady", j)
             yield ("mma", 0, "PV", j)
             if not self.tmut.oready_before_pv:
-                yield ("commit", 0, "VEmpty", j)
                 yield ("commit", 0, "OReady", j)
             if j + 2 < nt and not self.tmut.s_before_pv:
                 yield from issue_s(j + 2)
@@ -189,11 +189,10 @@ class TileModel(Model):
             return super()._exec_mma(a)
         self.queues[a].pop(0)
         if op[2] == "S":
-            _, _, _, j, s, slot = op
+            j = op[3]
             self._read_smem("Q", 0)
-            self._read_smem("K%d" % slot, (j, s))
-            if s > 0:
-                return
+            for s in range(K_SLICES):
+                self._read_smem("K%d" % ((K_SLICES * j + s) % K_SLOTS), (j, s))
             S = self.Sbuf[j & 1]
             if S["tag"] is not None:
                 if len(S["readers"]) != 4:
