@@ -38,7 +38,8 @@ namespace {
 constexpr int kSimWarps = 8;             // warps per CTA; 32 tokens per CTA
 constexpr int kWinWords = 4096;          // walk window: 131072 tokens (max_len <= 65536)
 constexpr int kWalkThreads = 256;
-constexpr int kStartBuf = 1024;          // chunk starts the walking thread lists before the CTA writes them
+constexpr int kStartBuf = 1024;          // chain entries the walking thread lists before the CTA writes them
+constexpr int kNodeCap = 8192;           // drops per window the walk tabulates (more: step by step)
 constexpr int kCompactThreads = 1024;
 
 __device__ __forceinline__ void to_float(const uint4& v, float* f, const __nv_bfloat16*) {
@@ -151,16 +152,92 @@ __global__ void __launch_bounds__(32 * kSimWarps)
   }
 }
 
+// Shared memory of the walk (dynamic: about 150 KB).
+struct WalkSmem {
+  uint32_t win[kWinWords];       // the window's drop bits
+  int nd[kWinWords + 1];         // nd[i]: first drop at or after word wb + i in the window, else kNone
+  int rank[kWinWords + 1];       // drops before word wb + i of the window
+  int node_pos[kNodeCap];        // the window's drops, ascending
+  int node_next[kNodeCap];       // walk from a chunk start at that drop: next drop that starts a chunk, or kEnd / kOut
+  int node_k[kNodeCap];          // forced starts (x + max_len, x + 2 max_len, ...) before it
+  int e_pos[kStartBuf];          // chain entries of this round: a start and its forced starts
+  int e_k[kStartBuf];
+  int e_pre[kStartBuf + 1];      // starts before entry e (exclusive prefix of e_k + 1)
+  int carry[kWalkThreads / 32];
+};
+
+constexpr int kNone = 0x7fffffff;
+constexpr int kEnd = -1;  // the walk reaches the end of the sequence
+constexpr int kOut = -2;  // the walk needs bits past the window
+
+// The walk's rule from a chunk start x, within the window: the next start is
+// the first drop in [x + min_len, x + max_len), else x + max_len (a forced
+// start) while that is inside the sequence.  Runs of forced starts are taken
+// in closed form: with no drop before f, every start x + k max_len below f is
+// forced.  Returns the first drop that becomes a start (>= 0), kEnd or kOut;
+// *forced counts the forced starts on the way and *last is the last start
+// reached (x itself, or its last forced start).
+__device__ int walk_from(const WalkSmem& S, int x, int wb, int n, bool full, int s1, int min_len, int max_len,
+                         int* forced, int* last) {
+  int k_forced = 0;
+  int result;
+  while (true) {
+    const long long clo = static_cast<long long>(x) + min_len;
+    if (clo >= s1) { result = kEnd; break; }
+    const long long xm = static_cast<long long>(x) + max_len;
+    const int chi = static_cast<int>(xm < s1 ? xm : s1);
+    if (((chi - 1) >> 5) >= wb + n) { result = kOut; break; }
+    // first drop at or after clo (none needed when min_len == max_len: the
+    // rule's interval is empty, and every start is forced)
+    int f = kNone;
+    if (clo < chi) {
+      const int wl = static_cast<int>(clo >> 5);
+      const uint32_t m = S.win[wl - wb] & (0xffffffffu << (clo & 31));
+      f = m != 0u ? (wl << 5) + __ffs(m) - 1 : S.nd[wl - wb + 1];
+    }
+    if (f < chi) { result = f; break; }
+    if (xm >= s1) { result = kEnd; break; }
+    if (f == kNone) {
+      if (full) {  // no drop up to the end: forced starts while below s1
+        k_forced += static_cast<int>((static_cast<long long>(s1) - 1 - x) / max_len);
+        x += static_cast<int>((static_cast<long long>(s1) - 1 - x) / max_len) * max_len;
+        result = kEnd;
+        break;
+      }
+      // no drop in the rest of the window: forced starts while their rule
+      // window stays inside it, then the walk needs the next window
+      // (at least the one forced start x + max_len, which is certain: no drop
+      // in [x + min_len, x + max_len) and x + max_len < s1; so every call
+      // that leaves the window has moved the walk on)
+      const long long room = (static_cast<long long>(wb + n) << 5) - x;
+      const int k = max(1, static_cast<int>(room / max_len) - 1);
+      x += k * max_len;
+      k_forced += k;
+      continue;
+    }
+    // f >= x + max_len: the starts x + max_len, ..., x + k max_len <= f are forced
+    const int k = (f - x) / max_len;
+    x += k * max_len;
+    k_forced += k;
+  }
+  *forced = k_forced;
+  *last = x;
+  return result;
+}
+
+// index of drop position f (a drop inside the window) in node_pos
+__device__ __forceinline__ int node_index(const WalkSmem& S, int f, int wb) {
+  const int wi = (f >> 5) - wb;
+  return S.rank[wi] + __popc(S.win[wi] & ((1u << (f & 31)) - 1u));
+}
+
 __global__ void __launch_bounds__(kWalkThreads)
     segment_walk_kernel(const uint32_t* __restrict__ drop, const int* __restrict__ cu_seqlens, int min_len,
                         int max_len, uint32_t* __restrict__ start_bits, uint32_t* status) {
-  __shared__ __align__(128) uint32_t win[kWinWords];
-  __shared__ int nd[kWinWords + 1];  // nd[i]: first drop at or after word wb + i (in the window), else kNone
-  __shared__ int s_carry[kWalkThreads / 32];
+  extern __shared__ __align__(128) unsigned char walk_smem_raw[];
+  WalkSmem& S = *reinterpret_cast<WalkSmem*>(walk_smem_raw);
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_starts[kStartBuf];  // chunk starts found by the walk, written out by the CTA
-  __shared__ int s_abort, s_b, s_done, s_nstarts;
-  constexpr int kNone = 0x7fffffff;
+  __shared__ int s_abort, s_b, s_done, s_ne, s_nodes;
   const int seq = blockIdx.x;
   const int s0 = cu_seqlens[seq], s1 = cu_seqlens[seq + 1];
   if (s1 <= s0) return;
@@ -176,6 +253,8 @@ __global__ void __launch_bounds__(kWalkThreads)
   __syncthreads();
   int b = s0;
   int wb = -1;  // first word held in the window (a multiple of 4: 16-byte copies)
+  int n = 0;
+  bool full = false;
   uint32_t phase = 0;
   while (true) {
     const int lo = b + min_len;
@@ -185,81 +264,172 @@ __global__ void __launch_bounds__(kWalkThreads)
       // [lo, hi) spans at most (max_len + 29) / 32 + 1 words and wb is at most
       // 3 words below lo's word, so the new window holds it
       wb = (lo >> 5) & ~3;
-      const int n = min(kWinWords, last_word + 1 - wb);
+      n = min(kWinWords, last_word + 1 - wb);
+      full = wb + n > last_word;
       const uint32_t bytes = static_cast<uint32_t>((n + 3) & ~3) * 4u;  // inside the 256-byte-aligned bitmap
       __syncthreads();  // every thread is done with the old window
       if (tid == 0) {
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(mbar, bytes);
-        bulk_load_1d(smem_u32(win), drop + wb, bytes, mbar);
+        bulk_load_1d(smem_u32(S.win), drop + wb, bytes, mbar);
       }
       const bool ok = mbar_wait(mbar, phase, &s_abort, status);
       phase ^= 1u;
       if (__syncthreads_or(!ok)) return;  // recorded in the status word
-      // nd = suffix minimum of each word's first drop: within each thread's
-      // run of words, then across threads (a suffix-min scan), then patched
+      // nd = suffix minimum of each word's first drop; rank = prefix count of
+      // drops: both within each thread's run of words, then across threads
       constexpr int kPer = kWinWords / kWalkThreads;
       const int i0 = tid * kPer, i1 = min(n, i0 + kPer);
-      int run = kNone;
+      int run = kNone, cnt = 0;
       for (int i = i1 - 1; i >= i0; --i) {
-        const uint32_t m = win[i];
+        const uint32_t m = S.win[i];
         if (m != 0u) run = ((wb + i) << 5) + __ffs(m) - 1;
-        nd[i] = run;
+        S.nd[i] = run;
+        cnt += __popc(m);
       }
       int suf = run;  // suffix minimum over threads tid .. (inclusive) in this warp
+      int incl = cnt;  // prefix sum over threads .. tid (inclusive) in this warp
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_down_sync(0xffffffffu, suf, o);
         if (lane + o < 32) suf = min(suf, v);
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
       }
-      if (lane == 0) s_carry[warp] = suf;
+      if (lane == 0) S.carry[warp] = suf;
+      if (lane == 31) S.e_pre[warp] = incl;  // per-warp drop totals (e_pre is free here)
       __syncthreads();
       int carry = __shfl_down_sync(0xffffffffu, suf, 1);
       if (lane == 31) carry = kNone;
-      for (int w = warp + 1; w < kWalkThreads / 32; ++w) carry = min(carry, s_carry[w]);
-      for (int i = i0; i < i1; ++i)
-        if (nd[i] == kNone) nd[i] = carry;
-      if (tid == 0) nd[n] = kNone;
+      for (int w = warp + 1; w < kWalkThreads / 32; ++w) carry = min(carry, S.carry[w]);
+      int before = incl - cnt;
+      for (int w = 0; w < warp; ++w) before += S.e_pre[w];
+      int total = 0;
+      for (int w = 0; w < kWalkThreads / 32; ++w) total += S.e_pre[w];
+      for (int i = i0; i < i1; ++i) {
+        if (S.nd[i] == kNone) S.nd[i] = carry;
+        S.rank[i] = before;
+        before += __popc(S.win[i]);
+      }
+      if (tid == 0) {
+        S.nd[n] = kNone;
+        S.rank[n] = total;
+        s_nodes = total;
+      }
+      __syncthreads();
+      const int nodes = s_nodes;
+      if (nodes <= kNodeCap) {
+        // the window's drops, then the walk's step from each of them
+        for (int i = i0; i < i1; ++i) {
+          uint32_t m = S.win[i];
+          int r = S.rank[i];
+          while (m != 0u) {
+            S.node_pos[r++] = ((wb + i) << 5) + __ffs(m) - 1;
+            m &= m - 1u;
+          }
+        }
+        __syncthreads();
+        for (int j = tid; j < nodes; j += kWalkThreads) {
+          int forced, last;
+          const int f = walk_from(S, S.node_pos[j], wb, n, full, s1, min_len, max_len, &forced, &last);
+          S.node_next[j] = f >= 0 ? node_index(S, f, wb) : f;
+          S.node_k[j] = forced;
+        }
+      }
       __syncthreads();
     }
     if (tid == 0) {
-      // the walk: two shared-memory loads per chunk
-      int cb = b, done = 0, ns = 0;
-      while (ns < kStartBuf) {
-        const int clo = cb + min_len;
-        if (clo >= s1) { done = 1; break; }
-        const int chi = min(cb + max_len, s1);
-        const int wl = clo >> 5;
-        if (((chi - 1) >> 5) >= wb + kWinWords) break;  // the window must move first
-        // both loads depend on wl only: issue them together
-        const uint32_t w = win[wl - wb];
-        const int beyond = nd[wl - wb + 1];
-        const uint32_t m = w & (0xffffffffu << (clo & 31));
-        const int f = m != 0u ? (wl << 5) + __ffs(m) - 1 : beyond;
-        int next;
-        if (f < chi) {
-          next = f;
-        } else if (cb + max_len < s1) {
-          next = cb + max_len;
-        } else {
-          done = 1;
-          break;
+      int ne = 0, done = 0, cb = b;
+      if (s_nodes <= kNodeCap) {
+        // the chain: from b to its first drop start, then one shared-memory
+        // step per drop start (its successor and forced starts are tabulated)
+        int forced, last;
+        int f = walk_from(S, b, wb, n, full, s1, min_len, max_len, &forced, &last);
+        S.e_pos[0] = b;
+        S.e_k[0] = forced;
+        ne = 1;
+        cb = last;
+        int j = f >= 0 ? node_index(S, f, wb) : f;
+        while (j >= 0 && ne < kStartBuf) {
+          const int pos = S.node_pos[j], k = S.node_k[j];
+          S.e_pos[ne] = pos;
+          S.e_k[ne] = k;
+          ++ne;
+          cb = pos + k * max_len;
+          j = S.node_next[j];
         }
-        s_starts[ns++] = next;
-        cb = next;
+        done = j == kEnd;
+      } else {
+        // too many drops to tabulate: the rule step by step, two
+        // shared-memory loads per chunk
+        while (ne < kStartBuf) {
+          const int clo = cb + min_len;
+          if (clo >= s1) { done = 1; break; }
+          const int chi = min(cb + max_len, s1);
+          if (((chi - 1) >> 5) >= wb + n) break;  // the window must move first
+          int f = kNone;  // first drop at or after clo (the interval is empty when min_len == max_len)
+          if (clo < chi) {
+            const int wl = clo >> 5;
+            const uint32_t m = S.win[wl - wb] & (0xffffffffu << (clo & 31));
+            f = m != 0u ? (wl << 5) + __ffs(m) - 1 : S.nd[wl - wb + 1];
+          }
+          int next;
+          if (f < chi) {
+            next = f;
+          } else if (cb + max_len < s1) {
+            next = cb + max_len;
+          } else {
+            done = 1;
+            break;
+          }
+          S.e_pos[ne] = next;
+          S.e_k[ne] = 0;
+          ++ne;
+          cb = next;
+        }
       }
       s_b = cb;
       s_done = done;
-      s_nstarts = ns;
+      s_ne = ne;
     }
     __syncthreads();
     b = s_b;
-    const int fin = s_done;
-    for (int i = tid; i < s_nstarts; i += kWalkThreads) {
-      const int p = s_starts[i];
-      atomicOr(start_bits + (p >> 5), 1u << (p & 31));
+    const int fin = s_done, ne = s_ne;
+    // set the starts: each entry's start and its forced starts, spread over
+    // the block by an exclusive prefix of (forced + 1)
+    {
+      constexpr int kPerE = kStartBuf / kWalkThreads;
+      int cnt = 0;
+      for (int e = tid * kPerE; e < min(ne, (tid + 1) * kPerE); ++e) cnt += S.e_k[e] + 1;
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (lane == 31) S.carry[warp] = incl;
+      __syncthreads();
+      int before = incl - cnt;
+      for (int w = 0; w < warp; ++w) before += S.carry[w];
+      int total = 0;
+      for (int w = 0; w < kWalkThreads / 32; ++w) total += S.carry[w];
+      for (int e = tid * kPerE; e < min(ne, (tid + 1) * kPerE); ++e) {
+        S.e_pre[e] = before;
+        before += S.e_k[e] + 1;
+      }
+      if (tid == 0) S.e_pre[ne] = total;
+      __syncthreads();
+      for (int t = tid; t < total; t += kWalkThreads) {
+        int lo_e = 0, hi_e = ne - 1;  // last entry with e_pre <= t
+        while (lo_e < hi_e) {
+          const int mid = (lo_e + hi_e + 1) >> 1;
+          if (S.e_pre[mid] <= t) lo_e = mid; else hi_e = mid - 1;
+        }
+        const int p = S.e_pos[lo_e] + (t - S.e_pre[lo_e]) * max_len;
+        atomicOr(start_bits + (p >> 5), 1u << (p & 31));
+      }
     }
-    __syncthreads();  // s_b, s_done and the start list are rewritten by the next round
+    __syncthreads();  // s_b, s_done and the entries are rewritten by the next round
     if (fin) break;
   }
 }
@@ -357,8 +527,11 @@ cudaError_t launch_segment(const void* k, int dtype, int total_tokens, int num_k
     }
     if (e != cudaSuccess) return e;
     if (num_seqs > 0) {
-      segment_walk_kernel<<<num_seqs, kWalkThreads, 0, stream>>>(drop, cu_seqlens, min_len, max_len, start_bits,
-                                                                 status);
+      constexpr int walk_smem = static_cast<int>(sizeof(WalkSmem));
+      e = cudaFuncSetAttribute(segment_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, walk_smem);
+      if (e != cudaSuccess) return e;
+      segment_walk_kernel<<<num_seqs, kWalkThreads, walk_smem, stream>>>(drop, cu_seqlens, min_len, max_len,
+                                                                         start_bits, status);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
