@@ -17,13 +17,18 @@
 //     per token ("drop": sim(t) < threshold) into a bitmap.  HBM-bound: every key row is read once from
 //     DRAM (the row before a warp's first token, read by the neighbouring warp
 //     too, hits in cache).
-//  2. segment_walk_kernel: one CTA per sequence.  The sequence's drop bits are
-//     brought into shared memory by a bulk copy, a window of kWinWords words at
-//     a time, and the CTA tabulates for every word the first drop at or after
-//     it (a suffix minimum).  One thread then walks the rule: from chunk start
+//  2. segment_walk_kernel: one CTA per sequence.  The rule: from chunk start
 //     b, the next start is the first drop in [b + min_len, b + max_len), else
-//     b + max_len: two shared-memory loads per chunk.  Chunk starts are set in
-//     a second bitmap.
+//     b + max_len.  The sequence's drop bits are brought into shared memory by
+//     a bulk copy, a window of kWinWords words at a time.  Every drop of the
+//     window is a possible chunk start, so the CTA lists them (ascending) and
+//     takes, in parallel, the rule's step from each: the next drop that
+//     becomes a start and the forced starts (x + max_len, x + 2 max_len, ...)
+//     before it, found by binary search in the list.  The drops reached from
+//     the window's first start are then found by pointer jumping (log2 of the
+//     drop count rounds), and every thread sets the starts of the drops it
+//     holds.  A window with more drops than the list holds is walked step by
+//     step by one thread instead.  Chunk starts are set in a second bitmap.
 //  3. segment_compact_kernel: one CTA turns the start bitmap into chunk_bounds
 //     (a block-wide scan of per-thread bit counts), then seq_chunk_ptr by binary
 //     search of each sequence's first token.
@@ -152,33 +157,45 @@ __global__ void __launch_bounds__(32 * kSimWarps)
   }
 }
 
-// Shared memory of the walk (dynamic: about 150 KB).
+// Shared memory of the walk (dynamic: about 180 KB).
 struct WalkSmem {
-  uint32_t win[kWinWords];       // the window's drop bits
-  int nd[kWinWords + 1];         // nd[i]: first drop at or after word wb + i in the window, else kNone
-  int rank[kWinWords + 1];       // drops before word wb + i of the window
-  int node_pos[kNodeCap];        // the window's drops, ascending
-  int node_next[kNodeCap];       // walk from a chunk start at that drop: next drop that starts a chunk, or kEnd / kOut
-  int node_k[kNodeCap];          // forced starts (x + max_len, x + 2 max_len, ...) before it
-  int e_pos[kStartBuf];          // chain entries of this round: a start and its forced starts
-  int e_k[kStartBuf];
-  int e_pre[kStartBuf + 1];      // starts before entry e (exclusive prefix of e_k + 1)
+  uint32_t win[kWinWords];            // the window's drop bits
+  int nd[kWinWords + 1];              // step-by-step walk only: first drop at or after word wb + i, else kNone
+  int node_pos[kNodeCap];             // the window's drops, ascending
+  int node_next[kNodeCap];            // walk from a chunk start at that drop: next drop start, or kEnd / kOut
+  int node_k[kNodeCap];               // forced starts (x + max_len, x + 2 max_len, ...) before it
+  int jump[kNodeCap];                 // pointer jumping: the node 2^r starts further on
+  unsigned char on_chain[kNodeCap];   // reached from the window's first start
+  int e_pos[kStartBuf];               // step-by-step walk: the starts it found this round
+  int warp_cnt[kWalkThreads / 32];
   int carry[kWalkThreads / 32];
 };
 
 constexpr int kNone = 0x7fffffff;
 constexpr int kEnd = -1;  // the walk reaches the end of the sequence
 constexpr int kOut = -2;  // the walk needs bits past the window
+constexpr int kNodesPerThread = kNodeCap / kWalkThreads;
+
+// first drop at or after x among the window's drops (ascending node_pos[0, nodes)):
+// its index, or nodes when there is none
+__device__ __forceinline__ int first_node_at_or_after(const WalkSmem& S, int nodes, long long x) {
+  int lo = 0, hi = nodes;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (S.node_pos[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
 
 // The walk's rule from a chunk start x, within the window: the next start is
 // the first drop in [x + min_len, x + max_len), else x + max_len (a forced
 // start) while that is inside the sequence.  Runs of forced starts are taken
 // in closed form: with no drop before f, every start x + k max_len below f is
-// forced.  Returns the first drop that becomes a start (>= 0), kEnd or kOut;
-// *forced counts the forced starts on the way and *last is the last start
-// reached (x itself, or its last forced start).
-__device__ int walk_from(const WalkSmem& S, int x, int wb, int n, bool full, int s1, int min_len, int max_len,
-                         int* forced, int* last) {
+// forced.  Returns the index of the first drop that becomes a start (>= 0),
+// kEnd or kOut; *forced counts the forced starts on the way and *last is the
+// last start reached (x itself, or its last forced start).
+__device__ int walk_from(const WalkSmem& S, int nodes, int x, int wb, int n, bool full, int s1, int min_len,
+                         int max_len, int* forced, int* last) {
   int k_forced = 0;
   int result;
   while (true) {
@@ -189,26 +206,26 @@ __device__ int walk_from(const WalkSmem& S, int x, int wb, int n, bool full, int
     if (((chi - 1) >> 5) >= wb + n) { result = kOut; break; }
     // first drop at or after clo (none needed when min_len == max_len: the
     // rule's interval is empty, and every start is forced)
-    int f = kNone;
+    int idx = nodes, f = kNone;
     if (clo < chi) {
-      const int wl = static_cast<int>(clo >> 5);
-      const uint32_t m = S.win[wl - wb] & (0xffffffffu << (clo & 31));
-      f = m != 0u ? (wl << 5) + __ffs(m) - 1 : S.nd[wl - wb + 1];
+      idx = first_node_at_or_after(S, nodes, clo);
+      if (idx < nodes) f = S.node_pos[idx];
     }
-    if (f < chi) { result = f; break; }
+    if (f < chi) { result = idx; break; }
     if (xm >= s1) { result = kEnd; break; }
     if (f == kNone) {
       if (full) {  // no drop up to the end: forced starts while below s1
-        k_forced += static_cast<int>((static_cast<long long>(s1) - 1 - x) / max_len);
-        x += static_cast<int>((static_cast<long long>(s1) - 1 - x) / max_len) * max_len;
+        const int k = static_cast<int>((static_cast<long long>(s1) - 1 - x) / max_len);
+        k_forced += k;
+        x += k * max_len;
         result = kEnd;
         break;
       }
       // no drop in the rest of the window: forced starts while their rule
-      // window stays inside it, then the walk needs the next window
-      // (at least the one forced start x + max_len, which is certain: no drop
-      // in [x + min_len, x + max_len) and x + max_len < s1; so every call
-      // that leaves the window has moved the walk on)
+      // window stays inside it (at least the one forced start x + max_len,
+      // which is certain: no drop in [x + min_len, x + max_len) and
+      // x + max_len < s1; so every call that leaves the window has moved the
+      // walk on), then the walk needs the next window
       const long long room = (static_cast<long long>(wb + n) << 5) - x;
       const int k = max(1, static_cast<int>(room / max_len) - 1);
       x += k * max_len;
@@ -225,10 +242,8 @@ __device__ int walk_from(const WalkSmem& S, int x, int wb, int n, bool full, int
   return result;
 }
 
-// index of drop position f (a drop inside the window) in node_pos
-__device__ __forceinline__ int node_index(const WalkSmem& S, int f, int wb) {
-  const int wi = (f >> 5) - wb;
-  return S.rank[wi] + __popc(S.win[wi] & ((1u << (f & 31)) - 1u));
+__device__ __forceinline__ void set_start(uint32_t* start_bits, int p) {
+  atomicOr(start_bits + (p >> 5), 1u << (p & 31));
 }
 
 __global__ void __launch_bounds__(kWalkThreads)
@@ -237,7 +252,7 @@ __global__ void __launch_bounds__(kWalkThreads)
   extern __shared__ __align__(128) unsigned char walk_smem_raw[];
   WalkSmem& S = *reinterpret_cast<WalkSmem*>(walk_smem_raw);
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_abort, s_b, s_done, s_ne, s_nodes;
+  __shared__ int s_abort, s_b, s_done, s_ne, s_nodes, s_first, s_forced;
   const int seq = blockIdx.x;
   const int s0 = cu_seqlens[seq], s1 = cu_seqlens[seq + 1];
   if (s1 <= s0) return;
@@ -248,7 +263,7 @@ __global__ void __launch_bounds__(kWalkThreads)
     s_abort = 0;
     mbar_init(mbar, 1);
     fence_mbar_init();
-    atomicOr(start_bits + (s0 >> 5), 1u << (s0 & 31));
+    set_start(start_bits, s0);
   }
   __syncthreads();
   int b = s0;
@@ -256,6 +271,7 @@ __global__ void __launch_bounds__(kWalkThreads)
   int n = 0;
   bool full = false;
   uint32_t phase = 0;
+  constexpr int kWarpWords = kWinWords / (kWalkThreads / 32);  // words of the window per warp
   while (true) {
     const int lo = b + min_len;
     if (lo >= s1) break;
@@ -276,117 +292,168 @@ __global__ void __launch_bounds__(kWalkThreads)
       const bool ok = mbar_wait(mbar, phase, &s_abort, status);
       phase ^= 1u;
       if (__syncthreads_or(!ok)) return;  // recorded in the status word
-      // nd = suffix minimum of each word's first drop; rank = prefix count of
-      // drops: both within each thread's run of words, then across threads
-      constexpr int kPer = kWinWords / kWalkThreads;
-      const int i0 = tid * kPer, i1 = min(n, i0 + kPer);
-      int run = kNone, cnt = 0;
-      for (int i = i1 - 1; i >= i0; --i) {
-        const uint32_t m = S.win[i];
-        if (m != 0u) run = ((wb + i) << 5) + __ffs(m) - 1;
-        S.nd[i] = run;
-        cnt += __popc(m);
+      // drops per warp: warp w holds words [w * kWarpWords, (w + 1) * kWarpWords),
+      // its lanes consecutive words (no bank conflicts)
+      const int w0 = warp * kWarpWords;
+      int cnt = 0;
+      for (int c = 0; c < kWarpWords; c += 32) {
+        const int i = w0 + c + lane;
+        if (i < n) cnt += __popc(S.win[i]);
       }
-      int suf = run;  // suffix minimum over threads tid .. (inclusive) in this warp
-      int incl = cnt;  // prefix sum over threads .. tid (inclusive) in this warp
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf = min(suf, v);
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      if (lane == 0) S.carry[warp] = suf;
-      if (lane == 31) S.e_pre[warp] = incl;  // per-warp drop totals (e_pre is free here)
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (lane == 0) S.warp_cnt[warp] = cnt;
       __syncthreads();
-      int carry = __shfl_down_sync(0xffffffffu, suf, 1);
-      if (lane == 31) carry = kNone;
-      for (int w = warp + 1; w < kWalkThreads / 32; ++w) carry = min(carry, S.carry[w]);
-      int before = incl - cnt;
-      for (int w = 0; w < warp; ++w) before += S.e_pre[w];
-      int total = 0;
-      for (int w = 0; w < kWalkThreads / 32; ++w) total += S.e_pre[w];
-      for (int i = i0; i < i1; ++i) {
-        if (S.nd[i] == kNone) S.nd[i] = carry;
-        S.rank[i] = before;
-        before += __popc(S.win[i]);
+      int base = 0, nodes = 0;
+      for (int w = 0; w < kWalkThreads / 32; ++w) {
+        if (w < warp) base += S.warp_cnt[w];
+        nodes += S.warp_cnt[w];
       }
-      if (tid == 0) {
-        S.nd[n] = kNone;
-        S.rank[n] = total;
-        s_nodes = total;
-      }
-      __syncthreads();
-      const int nodes = s_nodes;
       if (nodes <= kNodeCap) {
-        // the window's drops, then the walk's step from each of them
-        for (int i = i0; i < i1; ++i) {
-          uint32_t m = S.win[i];
-          int r = S.rank[i];
+        // the window's drops in ascending order: a warp prefix per 32 words
+        for (int c = 0; c < kWarpWords; c += 32) {
+          const int i = w0 + c + lane;
+          uint32_t m = i < n ? S.win[i] : 0u;
+          const int pc = __popc(m);
+          int incl = pc;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+          }
+          int r = base + incl - pc;
           while (m != 0u) {
             S.node_pos[r++] = ((wb + i) << 5) + __ffs(m) - 1;
             m &= m - 1u;
           }
+          base += __shfl_sync(0xffffffffu, incl, 31);
         }
         __syncthreads();
+        // the walk's step from a start at each drop
         for (int j = tid; j < nodes; j += kWalkThreads) {
           int forced, last;
-          const int f = walk_from(S, S.node_pos[j], wb, n, full, s1, min_len, max_len, &forced, &last);
-          S.node_next[j] = f >= 0 ? node_index(S, f, wb) : f;
+          S.node_next[j] = walk_from(S, nodes, S.node_pos[j], wb, n, full, s1, min_len, max_len, &forced, &last);
           S.node_k[j] = forced;
+        }
+      } else {
+        // too many drops to tabulate: nd = suffix minimum of each word's first
+        // drop, for the step-by-step walk (within each thread's run of words,
+        // then across threads)
+        constexpr int kPer = kWinWords / kWalkThreads;
+        const int i0 = tid * kPer, i1 = min(n, i0 + kPer);
+        int run = kNone;
+        for (int i = i1 - 1; i >= i0; --i) {
+          const uint32_t m = S.win[i];
+          if (m != 0u) run = ((wb + i) << 5) + __ffs(m) - 1;
+          S.nd[i] = run;
+        }
+        int suf = run;  // suffix minimum over threads tid .. (inclusive) in this warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_down_sync(0xffffffffu, suf, o);
+          if (lane + o < 32) suf = min(suf, v);
+        }
+        if (lane == 0) S.carry[warp] = suf;
+        __syncthreads();
+        int carry = __shfl_down_sync(0xffffffffu, suf, 1);
+        if (lane == 31) carry = kNone;
+        for (int w = warp + 1; w < kWalkThreads / 32; ++w) carry = min(carry, S.carry[w]);
+        for (int i = i0; i < i1; ++i)
+          if (S.nd[i] == kNone) S.nd[i] = carry;
+        if (tid == 0) S.nd[n] = kNone;
+      }
+      if (tid == 0) s_nodes = nodes;
+      __syncthreads();
+    }
+    const int nodes = s_nodes;
+    if (nodes <= kNodeCap) {
+      // the chain from b: its first drop start (thread 0), then every drop
+      // start reached from it, found by pointer jumping (round r marks the
+      // nodes 2^r .. 2^(r+1) - 1 steps on), all in parallel
+      if (tid == 0) {
+        int forced, last;
+        const int f = walk_from(S, nodes, b, wb, n, full, s1, min_len, max_len, &forced, &last);
+        s_first = f;
+        s_forced = forced;
+        s_b = last;
+        s_done = f == kEnd;
+      }
+      __syncthreads();
+      const int first = s_first;
+      for (int k = 1 + tid; k <= s_forced; k += kWalkThreads) set_start(start_bits, b + k * max_len);
+      if (first >= 0) {
+        for (int j = tid; j < nodes; j += kWalkThreads) {
+          S.on_chain[j] = j == first;
+          S.jump[j] = S.node_next[j];
+        }
+        __syncthreads();
+        for (int span = 1; span <= nodes; span <<= 1) {
+          int nxt[kNodesPerThread];
+#pragma unroll
+          for (int q = 0; q < kNodesPerThread; ++q) {
+            const int j = tid + q * kWalkThreads;
+            nxt[q] = kEnd;
+            if (j < nodes) {
+              const int t = S.jump[j];
+              if (t >= 0) {
+                if (S.on_chain[j]) S.on_chain[t] = 1;  // every node written here is on the chain
+                nxt[q] = S.jump[t];
+              } else {
+                nxt[q] = t;
+              }
+            }
+          }
+          __syncthreads();
+#pragma unroll
+          for (int q = 0; q < kNodesPerThread; ++q) {
+            const int j = tid + q * kWalkThreads;
+            if (j < nodes) S.jump[j] = nxt[q];
+          }
+          __syncthreads();
+        }
+        // the starts: every node on the chain and its forced starts; the one
+        // whose step leaves the chain (end of sequence or of window) sets b
+        for (int j = tid; j < nodes; j += kWalkThreads) {
+          if (!S.on_chain[j]) continue;
+          const int pos = S.node_pos[j], k = S.node_k[j];
+          for (int q = 0; q <= k; ++q) set_start(start_bits, pos + q * max_len);
+          const int nx = S.node_next[j];
+          if (nx < 0) {
+            s_b = pos + k * max_len;
+            s_done = nx == kEnd;
+          }
         }
       }
       __syncthreads();
+      b = s_b;
+      if (s_done) break;
+      __syncthreads();  // s_b and s_done are rewritten by the next round
+      continue;
     }
+    // step by step, two shared-memory loads per chunk
     if (tid == 0) {
       int ne = 0, done = 0, cb = b;
-      if (s_nodes <= kNodeCap) {
-        // the chain: from b to its first drop start, then one shared-memory
-        // step per drop start (its successor and forced starts are tabulated)
-        int forced, last;
-        int f = walk_from(S, b, wb, n, full, s1, min_len, max_len, &forced, &last);
-        S.e_pos[0] = b;
-        S.e_k[0] = forced;
-        ne = 1;
-        cb = last;
-        int j = f >= 0 ? node_index(S, f, wb) : f;
-        while (j >= 0 && ne < kStartBuf) {
-          const int pos = S.node_pos[j], k = S.node_k[j];
-          S.e_pos[ne] = pos;
-          S.e_k[ne] = k;
-          ++ne;
-          cb = pos + k * max_len;
-          j = S.node_next[j];
+      while (ne < kStartBuf) {
+        const int clo = cb + min_len;
+        if (clo >= s1) { done = 1; break; }
+        const int chi = min(cb + max_len, s1);
+        if (((chi - 1) >> 5) >= wb + n) break;  // the window must move first
+        int f = kNone;  // first drop at or after clo (the interval is empty when min_len == max_len)
+        if (clo < chi) {
+          const int wl = clo >> 5;
+          const uint32_t m = S.win[wl - wb] & (0xffffffffu << (clo & 31));
+          f = m != 0u ? (wl << 5) + __ffs(m) - 1 : S.nd[wl - wb + 1];
         }
-        done = j == kEnd;
-      } else {
-        // too many drops to tabulate: the rule step by step, two
-        // shared-memory loads per chunk
-        while (ne < kStartBuf) {
-          const int clo = cb + min_len;
-          if (clo >= s1) { done = 1; break; }
-          const int chi = min(cb + max_len, s1);
-          if (((chi - 1) >> 5) >= wb + n) break;  // the window must move first
-          int f = kNone;  // first drop at or after clo (the interval is empty when min_len == max_len)
-          if (clo < chi) {
-            const int wl = clo >> 5;
-            const uint32_t m = S.win[wl - wb] & (0xffffffffu << (clo & 31));
-            f = m != 0u ? (wl << 5) + __ffs(m) - 1 : S.nd[wl - wb + 1];
-          }
-          int next;
-          if (f < chi) {
-            next = f;
-          } else if (cb + max_len < s1) {
-            next = cb + max_len;
-          } else {
-            done = 1;
-            break;
-          }
-          S.e_pos[ne] = next;
-          S.e_k[ne] = 0;
-          ++ne;
-          cb = next;
+        int next;
+        if (f < chi) {
+          next = f;
+        } else if (cb + max_len < s1) {
+          next = cb + max_len;
+        } else {
+          done = 1;
+          break;
         }
+        S.e_pos[ne++] = next;
+        cb = next;
       }
       s_b = cb;
       s_done = done;
@@ -394,42 +461,9 @@ __global__ void __launch_bounds__(kWalkThreads)
     }
     __syncthreads();
     b = s_b;
-    const int fin = s_done, ne = s_ne;
-    // set the starts: each entry's start and its forced starts, spread over
-    // the block by an exclusive prefix of (forced + 1)
-    {
-      constexpr int kPerE = kStartBuf / kWalkThreads;
-      int cnt = 0;
-      for (int e = tid * kPerE; e < min(ne, (tid + 1) * kPerE); ++e) cnt += S.e_k[e] + 1;
-      int incl = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      if (lane == 31) S.carry[warp] = incl;
-      __syncthreads();
-      int before = incl - cnt;
-      for (int w = 0; w < warp; ++w) before += S.carry[w];
-      int total = 0;
-      for (int w = 0; w < kWalkThreads / 32; ++w) total += S.carry[w];
-      for (int e = tid * kPerE; e < min(ne, (tid + 1) * kPerE); ++e) {
-        S.e_pre[e] = before;
-        before += S.e_k[e] + 1;
-      }
-      if (tid == 0) S.e_pre[ne] = total;
-      __syncthreads();
-      for (int t = tid; t < total; t += kWalkThreads) {
-        int lo_e = 0, hi_e = ne - 1;  // last entry with e_pre <= t
-        while (lo_e < hi_e) {
-          const int mid = (lo_e + hi_e + 1) >> 1;
-          if (S.e_pre[mid] <= t) lo_e = mid; else hi_e = mid - 1;
-        }
-        const int p = S.e_pos[lo_e] + (t - S.e_pre[lo_e]) * max_len;
-        atomicOr(start_bits + (p >> 5), 1u << (p & 31));
-      }
-    }
-    __syncthreads();  // s_b, s_done and the entries are rewritten by the next round
+    const int fin = s_done;
+    for (int e = tid; e < s_ne; e += kWalkThreads) set_start(start_bits, S.e_pos[e]);
+    __syncthreads();  // s_b, s_done and the start list are rewritten by the next round
     if (fin) break;
   }
 }
