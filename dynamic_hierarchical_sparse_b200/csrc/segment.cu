@@ -313,6 +313,7 @@ __global__ void __launch_bounds__(kWalkThreads)
         for (int c = 0; c < kWarpWords; c += 32) {
           const int i = w0 + c + lane;
           uint32_t m = i < n ? S.win[i] : 0u;
+          if (!__any_sync(0xffffffffu, m != 0u)) continue;  // no drop in these 32 words
           const int pc = __popc(m);
           int incl = pc;
 #pragma unroll
@@ -390,6 +391,7 @@ __global__ void __launch_bounds__(kWalkThreads)
           int nxt[kNodesPerThread];
 #pragma unroll
           for (int q = 0; q < kNodesPerThread; ++q) {
+            if (q * kWalkThreads >= nodes) break;  // the same for every thread
             const int j = tid + q * kWalkThreads;
             nxt[q] = kEnd;
             if (j < nodes) {
@@ -405,6 +407,7 @@ __global__ void __launch_bounds__(kWalkThreads)
           __syncthreads();
 #pragma unroll
           for (int q = 0; q < kNodesPerThread; ++q) {
+            if (q * kWalkThreads >= nodes) break;
             const int j = tid + q * kWalkThreads;
             if (j < nodes) S.jump[j] = nxt[q];
           }
