@@ -557,7 +557,8 @@ def bench_gpu(args):
                             "plan + attention and copy-out of consecutive steps overlap on three streams "
                             "(three device buffer sets)"},
         # per step: chunk reduce (Q and K in one launch), [group sum,] similarity, select, attention
-        "gpu_launches": (5 if args.kv_plan else 4) * args.steps,
+        # reduce, similarity, (group sum,) select; the f16 copy of V (bf16) and attention
+        "gpu_launches": ((5 if args.kv_plan else 4) + (1 if spec.dtype == "bf16" else 0)) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1:
@@ -792,7 +793,7 @@ def bench_online_chunking(args):
                    "rule": {"threshold": rule.threshold, "min_len": rule.min_len, "max_len": rule.max_len},
                    "num_chunks": int(hb.shape[0] - 1), "budget": _budget_str(inp.budget)},
         "ms_segment_and_readback": part[0], "ms_plan": part[1], "ms_attention": part[2],
-        "gpu_launches": 7 * args.steps,  # segment 3, plan 3, attention 1 per step
+        "gpu_launches": 8 * args.steps,  # segment 3, plan 3, f16 copy of V 1, attention 1 per step
         "clocks": clk,
     }), flush=True)
 

@@ -146,13 +146,24 @@ dhsa_status run_plan(const void* q, const void* k, const dhsa_problem* p, const 
   return run_select(scores, p, budget, row_ptr, col, status, st);
 }
 
+// Bytes of the attention workspace: the status word and the work-item
+// counter, then (bf16) the f16 copy of V that the P V products read.
+size_t attention_ws_bytes(const dhsa_problem* p) {
+  size_t b = kStatusBytes;
+  if (p->dtype == DHSA_BF16)
+    b += align_up(static_cast<size_t>(p->total_tokens) * p->num_kv_heads * p->head_dim * 2);
+  return b;
+}
+
 // Step 4 after validation; plan_group = query heads per plan row.
 dhsa_status run_attention(const void* q, const void* k, const void* v, const dhsa_problem* p,
                           const int32_t* row_ptr, const int32_t* col, int64_t nnz, int plan_group, float scale,
                           void* out, void* workspace, size_t workspace_bytes, cudaStream_t st) {
   if (nnz < static_cast<int64_t>(p->num_q_heads / plan_group) * p->num_chunks || nnz > INT32_MAX)
     return DHSA_ERR_INVALID_ARG;  // >= diagonal per row
-  if (workspace == nullptr || workspace_bytes < kStatusBytes) return DHSA_ERR_WORKSPACE;
+  if (workspace == nullptr || workspace_bytes < attention_ws_bytes(p) ||
+      (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return DHSA_ERR_WORKSPACE;
   if (p->total_tokens == 0 || p->num_chunks == 0) return DHSA_OK;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || row_ptr == nullptr || col == nullptr)
     return DHSA_ERR_INVALID_ARG;
@@ -168,10 +179,15 @@ dhsa_status run_attention(const void* q, const void* k, const void* v, const dhs
                                             p->num_kv_heads, p->head_dim, plan_group, scale,
                                             static_cast<float*>(out), status, st));
   }
+  // V in f16 for the P V products (P is f16 too: see the kernels)
+  void* v16 = static_cast<unsigned char*>(workspace) + kStatusBytes;
+  const long long v_elems = static_cast<long long>(p->total_tokens) * p->num_kv_heads * p->head_dim;
+  if (cudaError_t e = launch_v_to_f16(v, v16, v_elems, status, st); e != cudaSuccess) return cuda_status(e);
   AttnBf16Args a;
   a.q = q;
   a.k = k;
   a.v = v;
+  a.v16 = v16;
   a.out = out;
   a.bounds = p->chunk_bounds;
   a.row_ptr = row_ptr;
@@ -341,7 +357,7 @@ dhsa_status dhsa_attention_workspace_size(const dhsa_problem* p, size_t* bytes) 
   dhsa_status s = check_problem(p);
   if (s != DHSA_OK) return s;
   if (bytes == nullptr) return DHSA_ERR_INVALID_ARG;
-  *bytes = kStatusBytes;
+  *bytes = attention_ws_bytes(p);
   return DHSA_OK;
 }
 

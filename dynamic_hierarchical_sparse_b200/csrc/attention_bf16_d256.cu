@@ -18,8 +18,9 @@
 //   S_0, S_1  columns [0, 128) and [128, 256): S = Q K^T, double-buffered, so
 //             QK^T of tile j+1 runs on the tensor core while the softmax
 //             turns S(j) into P(j);
-//   P(j)      bf16, two per column, written by the softmax over the first 64
-//             columns of S(j%2): the A operand of O += P V straight from TMEM,
+//   P(j)      f16, two per column, written by the softmax over the first 64
+//             columns of S(j%2): the A operand of O += P V straight from TMEM
+//             (B: an f16 copy of V, made before the launch),
 //             so PV is one M=128, N=256 (= d) MMA per 16 keys, the tensor
 //             core's full-rate shape, with no P traffic through shared memory;
 //   O         columns [256, 512).
@@ -59,7 +60,7 @@ constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr uint32_t kTmemCols = 512;
 // O is rescaled whenever a warp's running max grows, so the largest weight
-// of a row is exp2(0) = 1, exact in bf16 (a lagging max would leave it rounded,
+// of a row is exp2(0) = 1, exact (a lagging max would leave it rounded,
 // and that rounding would reach O directly).
 constexpr float kRescaleLog2 = 0.0f;
 constexpr int kSlices = kD / 64;        // 64-column slices of a Q / K / V row
@@ -139,6 +140,15 @@ struct KeyTiles {
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// P as an f16 pair: the weights lie in [0, 1], where f16 keeps 11 significant
+// bits against bf16's 8, so rounding them perturbs O by at most 2^-12 max|V|
+// (2^-9 max|V| in bf16, which at |O| in [4, 8) adds to the output's own
+// rounding of up to 2^-6 and can pass a 2e-2 error bound).
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
@@ -323,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, kD, 1);
+      constexpr uint32_t idesc_o = idesc_f16_f32(kBM, kD, 1);  // P and V in f16
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, status);
       tc_fence_after();
       // S(j) = Q K(j)^T into buffer j % 2: one wait for the whole tile
@@ -443,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), scale2, shift2), x0, x1);
         const float e0 = ex2_approx(x0);
         const float e1 = ex2_approx(x1);
-        pk[c / 2] = pack_bf16(e0, e1);
+        pk[c / 2] = pack_f16(e0, e1);
         ps2[(c / 2) & 1] = f2_add(ps2[(c / 2) & 1], f2_pack(e0, e1));
       }
       // P(j) over the first 64 columns of S(j % 2) (its S values are in registers)
@@ -537,7 +547,7 @@ cudaError_t launch_attention_d256(const AttnBf16Args& a, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   if (encode_qkv_map(&mq, a.q, a.num_q_heads, kD, a.total_tokens, kBM) != CUDA_SUCCESS ||
       encode_qkv_map(&mk, a.k, a.num_kv_heads, kD, a.total_tokens, kBN) != CUDA_SUCCESS ||
-      encode_qkv_map(&mv, a.v, a.num_kv_heads, kD, a.total_tokens, kBN) != CUDA_SUCCESS)
+      encode_qkv_map(&mv, a.v16, a.num_kv_heads, kD, a.total_tokens, kBN, true) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   cudaError_t e =
       cudaFuncSetAttribute(attention_d256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

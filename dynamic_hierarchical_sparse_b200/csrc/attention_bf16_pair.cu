@@ -39,8 +39,10 @@
 // sub-partition's 16K); the third warpgroup then hands registers back
 // (setmaxnreg.dec to 56) and the softmax warpgroups take them (224), enough to
 // hold a whole 128-column row of S without spilling.
-// TMEM (512 columns): S_a at [128a, 128a+128); P_a (bf16, two per column) is
-// written over the first 64 columns of S_a and is the A operand of O_a += P_a V;
+// TMEM (512 columns): S_a at [128a, 128a+128); P_a (f16, two per column) is
+// written over the first 64 columns of S_a and is the A operand of O_a += P_a V
+// (B: an f16 copy of V, made before the launch; both operands of one MMA are
+// of one type);
 // O_a at [256 + a*D, 256 + (a+1)*D).  The tensor pipe takes
 //   PV_0(t), S_0(t+1), PV_1(t), S_1(t+1), PV_0(t+1), ...
 // so while one warpgroup turns S into P the tensor core works for the other.
@@ -83,9 +85,9 @@ constexpr int kRangeCap = 96;  // runs cached per item slot in shared memory; mo
 constexpr int kItemUsers = 11;  // item-slot releases: producer, two MMA threads, eight softmax warps
 constexpr int kVStages = 3;     // V ring depth (K uses 2)
 // O is rescaled whenever a warp's running max grows (threshold 0 in log2
-// units): the row's largest weight is then exp2(0) = 1, exact in bf16.  A lazy
+// units): the row's largest weight is then exp2(0) = 1, exact.  A lazy
 // threshold (2^8) let the running max lag, so the largest weight was rounded
-// to bf16 (2^-9 relative) and that rounding reached O directly: 0.026 of error
+// (to bf16 then, 2^-9 relative) and that rounding reached O directly: 0.026 of error
 // at |O| = 4.4 at 128K, against 0.017 with every growth rescaled, for about
 // 4 % of attention time.
 constexpr float kRescaleLog2 = 0.0f;
@@ -206,6 +208,15 @@ struct TileWalk {
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// P as an f16 pair: the weights lie in [0, 1], where f16 keeps 11 significant
+// bits against bf16's 8, so rounding them perturbs O by at most 2^-12 max|V|
+// (2^-9 max|V| in bf16, which at |O| in [4, 8) adds to the output's own
+// rounding of up to 2^-6 and can pass a 2e-2 error bound).
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
@@ -506,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int a = warp - kMmaWarp;
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 1);
+      constexpr uint32_t idesc_o = idesc_f16_f32(kBM, D, 1);  // P and V in f16
       const uint32_t qbase = sbase + C::kOffQ + a * C::kQBytes;
       auto issue_s = [&](int tg) {
         const uint32_t kbase = sbase + C::kOffK + (tg & 1) * C::kKVBytes;
@@ -690,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
       const uint64_t shift2 = f2_pack(-m_use, -m_use);
       uint32_t pk[kBN / 2];
-      // P = exp2(s * scale - m) for columns [cb, cb + 64), packed to bf16 pairs
+      // P = exp2(s * scale - m) for columns [cb, cb + 64), packed to f16 pairs
       auto exp_cols = [&](int cb) {
 #pragma unroll
         for (int c = cb; c < cb + kBN / 2; c += 2) {
@@ -707,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ps2[(c / 2) & 1] = f2_add(ps2[(c / 2) & 1], f2_pack(e0, e1));
           else
             ps[(c / 2) & 3] += e0 + e1;
-          pk[c / 2] = pack_bf16(e0, e1);
+          pk[c / 2] = pack_f16(e0, e1);
         }
       };
       // O is rescaled before PV(t) accumulates into it; PV(t-1) is done, since
@@ -816,7 +827,7 @@ cudaError_t launch_attention_pair_dim(const AttnBf16Args& a, cudaStream_t stream
   CUtensorMap mq, mk, mv;
   if (encode_qkv_map(&mq, a.q, a.num_q_heads, D, a.total_tokens, kBM) != CUDA_SUCCESS ||
       encode_qkv_map(&mk, a.k, a.num_kv_heads, D, a.total_tokens, kBN) != CUDA_SUCCESS ||
-      encode_qkv_map(&mv, a.v, a.num_kv_heads, D, a.total_tokens, kBN) != CUDA_SUCCESS)
+      encode_qkv_map(&mv, a.v16, a.num_kv_heads, D, a.total_tokens, kBN, true) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   auto kern = attention_pair_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -280,6 +281,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int b_mn_maj
   return (1u << 4)                              // D format: f32
          | (1u << 7)                            // A format: bf16
          | (1u << 10)                           // B format: bf16
+         | (static_cast<uint32_t>(b_mn_major) << 16)
+         | (static_cast<uint32_t>(n >> 3) << 17)
+         | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Instruction descriptor of kind::f16 with f16 A/B and fp32 D (format code 0
+// for both operands): the P V product, P and the copy of V in f16.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, int b_mn_major) {
+  return (1u << 4)  // D format: f32; A and B format: f16
          | (static_cast<uint32_t>(b_mn_major) << 16)
          | (static_cast<uint32_t>(n >> 3) << 17)
          | (static_cast<uint32_t>(m >> 4) << 24);

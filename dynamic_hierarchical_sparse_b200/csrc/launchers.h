@@ -52,6 +52,7 @@ struct AttnBf16Args {
   const void* q;
   const void* k;
   const void* v;
+  const void* v16;  // f16 copy of v (launch_v_to_f16), the B operand of the P V product
   void* out;
   const int* bounds;
   const int* row_ptr;
@@ -73,7 +74,11 @@ cudaError_t launch_attention_pair(const AttnBf16Args& a, cudaStream_t stream);
 // head_dim 256: one query tile per CTA, 128-key tiles, S double-buffered and P in TMEM.
 cudaError_t launch_attention_d256(const AttnBf16Args& a, cudaStream_t stream);
 // TMA view of a packed THD bf16 tensor (see attention_bf16.cu).
-CUresult encode_qkv_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows);
+CUresult encode_qkv_map(CUtensorMap* map, const void* base, int heads, int head_dim, int tokens, int box_rows,
+                        bool f16 = false);
+// v (bf16, n elements, n a multiple of 8) -> v16 (f16), exact for |v| <= 65504;
+// larger magnitudes are reported (kDevCheck).
+cudaError_t launch_v_to_f16(const void* v, void* v16, long long n, uint32_t* status, cudaStream_t stream);
 
 // Online chunking (three launches: adjacent-key similarity bits, a walk per
 // sequence, compaction).  drop and start_bits: ceil(T / 32) words each.

@@ -180,8 +180,14 @@ DHSA_API dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem*
  * accumulation and an fp32 online softmax; fp32 runs an fp32 kernel.
  *   q, k, v  device, THD, `dtype`; out device [T, Hq, d] in `dtype`
  *   row_ptr, col: a plan as written by dhsa_plan / dhsa_topk_select
- * Workspace: dhsa_attention_workspace_size bytes: the status word and the
- * work-item counter of the persistent bf16 kernel, both reset by each call.
+ * Workspace: dhsa_attention_workspace_size bytes, 256-byte aligned: the status
+ * word and the work-item counter of the persistent bf16 kernel, both reset by
+ * each call, then (bf16 problems) an f16 copy of v, T*Hkv*d*2 bytes, written by
+ * each call: the tensor cores take the softmax weights P and V in f16 (11
+ * significant bits for P in [0, 1] against bf16's 8, which keeps the weights'
+ * rounding under 2^-12 max|v|).  A |v| above 65504 (or NaN) has no f16
+ * counterpart: it is saturated and reported as DHSA_ERR_DEVICE_CHECK through
+ * dhsa_workspace_status.
  * A workspace serves one call at a time: calls that may overlap on the GPU
  * (other streams) need workspaces of their own. */
 DHSA_API dhsa_status dhsa_attention_workspace_size(const dhsa_problem* p, size_t* bytes);

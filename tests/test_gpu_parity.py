@@ -351,6 +351,29 @@ def test_empty_sequence_in_batch():
     attention_gate(out, want, torch.bfloat16)
 
 
+@pytest.mark.parametrize("d", [128, 256])
+def test_v_outside_f16_range_is_reported(d):
+    """The bf16 kernels read an f16 copy of V (P V in f16): a V magnitude above
+    65504 has no f16 counterpart and is reported (DHSA_ERR_DEVICE_CHECK); the
+    next call with a V in range runs clean and correct."""
+    inp = W.random_problem(11, [600], 2, 1, d, "bf16", 40, 160, W.Budget.topk(2))
+    q, k, v, prob = to_device(inp)
+    plan = api.plan(q, k, prob, inp.budget, check=True)
+    attn = api.Attention(prob, q.device)
+    out = torch.empty_like(q)
+    bad = v.clone()
+    bad[123, 0, 7] = 1.0e5
+    attn(q, k, bad, plan, out)
+    torch.cuda.synchronize()
+    assert attn.status() == 6
+    attn(q, k, v, plan, out)
+    torch.cuda.synchronize()
+    assert attn.status() == 0
+    want = O.attention_gather(inp.q, inp.k, inp.v, inp.chunk_bounds, plan.row_ptr.cpu().numpy(),
+                              plan.col.cpu().numpy())
+    attention_gate(out, want, torch.bfloat16)
+
+
 def test_timeout_path_reports_and_context_survives():
     assert api.selftest_timeout(20000) == 5  # DHSA_ERR_TIMEOUT
     inp = _case("d128_diag_only")

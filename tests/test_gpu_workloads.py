@@ -153,8 +153,9 @@ def test_select_microbench_rows():
 
 def test_memory_beyond_inputs_is_the_workspace():
     """At the 32K shape the memory a layer call allocates beyond Q/K/V/O is the
-    library's stated workspace and plan (O(T*H*d/L + H*n^2)), a few percent of
-    the inputs: no [T, T] object is ever materialised."""
+    library's stated workspace and plan (O(T*H*d/L + H*n^2), plus the f16 copy
+    of V that the bf16 attention reads, T*Hkv*d*2 bytes): no [T, T] object is
+    ever materialised."""
     import bench
 
     rep = bench.memory_report(W.LLAMA_32K)
@@ -162,5 +163,8 @@ def test_memory_beyond_inputs_is_the_workspace():
     print(rep)
     # torch's caching allocator rounds each block up to 2 MiB granularity at most
     assert rep["measured_peak_extra_bytes"] <= stated + 3 * (2 << 20)
-    assert rep["measured_peak_extra_bytes"] <= 0.05 * rep["qkvo_bytes"]
-    assert rep["measured_peak_extra_bytes"] < rep["dense_scores_bf16_bytes"] / 1000
+    spec = W.LLAMA_32K
+    v16 = spec.total_tokens * spec.num_kv_heads * spec.head_dim * 2
+    assert rep["measured_peak_extra_bytes"] <= v16 + 0.05 * rep["qkvo_bytes"]
+    # beyond the copy of V (linear in T), what remains is tiny against any [Hq, T, T] object
+    assert rep["measured_peak_extra_bytes"] - v16 < rep["dense_scores_bf16_bytes"] / 1000

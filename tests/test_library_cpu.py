@@ -90,7 +90,12 @@ def test_workspace_sizes():
     ws = p.plan_workspace_bytes(W.Budget.topk(4))
     need = 256 + (8 * n * 128 + 2 * n * 128 + 8 * n * n) * 4
     assert need <= ws <= need + 4 * 256
-    assert p.attention_workspace_bytes() >= 256
+    # bf16: the status words, then an f16 copy of V (T * Hkv * d * 2 bytes, 256-byte aligned)
+    v16 = 2048 * 2 * 128 * 2
+    assert p.attention_workspace_bytes() == 256 + v16
+    # fp32 needs no copy
+    inp32 = W.random_problem(0, [2048], 8, 2, 128, "f32", 64, 256, W.Budget.topk(4))
+    assert _problem(inp32).attention_workspace_bytes() == 256
 
 
 def test_per_kv_head_plan_sizes():
@@ -176,7 +181,14 @@ def test_entry_points_reject_before_launch():
     # misaligned q
     assert L.dhsa_attention(ctypes.c_void_p(17), ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(),
                             ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ctypes.c_float(0.0),
-                            ctypes.c_void_p(16), ws, 256, null) == 1
+                            ctypes.c_void_p(16), ws, 1 << 30, null) == 1
+    # a workspace without room for the f16 copy of V, or not 256-byte aligned
+    assert L.dhsa_attention(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(),
+                            ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ctypes.c_float(0.0),
+                            ctypes.c_void_p(16), ws, p.attention_workspace_bytes() - 1, null) == 3
+    assert L.dhsa_attention(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(),
+                            ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ctypes.c_float(0.0),
+                            ctypes.c_void_p(16), ctypes.c_void_p(272), 1 << 30, null) == 3
     # missing workspace
     assert L.dhsa_attention(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), p.ref(),
                             ctypes.c_void_p(16), ctypes.c_void_p(16), nnz, ctypes.c_float(0.0),
