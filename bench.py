@@ -46,8 +46,8 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # keeps the SHA-256 of that source (attention_bf16_pair.cu + common.cuh), and
 # any other source reports traffic as null.
 ATTN_TRAFFIC_CAPTURE = {
-    "bytes": 10.48e9,  # 9.44 GB read + 1.04 GB written
-    "source_sha256": "5362b0cea2af71ed7401ddaa5ef1135640c8d70b58ff4dfce32b384d0f4d0746",
+    "bytes": 10.466e9,  # 9.427 GB read + 1.040 GB written
+    "source_sha256": "5e739af4ab8cc692fea69f54f4e1d2c3212a34bfc245f3bb1b1182e4f61a703e",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:attention_pair -s 1 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-micro"),
 }
@@ -72,19 +72,27 @@ def _peaks():
 
 
 def tensor_peak(peaks, clk):
-    """The bf16 peak a kernel timed in this run is held against, chosen from
-    the SM clock sampled during the timed region: the burst figure (a GEMM
-    timed alone, at full clock) when the run's median clock is within 5 % of
-    the maximum, else the sustained figure (a seconds-long loop under the
-    power cap).  Returns (peak, kind)."""
+    """The bf16 peak a kernel timed in this run is held against, from the SM
+    clock sampled during the timed region: the burst figure (a GEMM timed
+    alone at the maximum clock) scaled by this run's median clock over the
+    maximum, since tensor throughput follows the clock, and never below the
+    sustained figure (a seconds-long loop under the power cap, at its lower
+    clock).  At the maximum clock this is the burst figure itself.  Returns
+    (peak, kind)."""
     sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz") or peaks.get("sm_max_mhz")
-    if sm is not None and smax and sm < 0.95 * smax:
-        return peaks["bf16_tflops_sustained"], ("%s bf16 dense, sustained (this run's median SM clock %.0f MHz is "
-                                                "below the maximum %.0f MHz)" % (peaks["source"], sm, smax))
-    return peaks["bf16_tflops"], ("%s bf16 dense, burst (this run's median SM clock %s MHz is the maximum; the "
-                                  "sustained figure was taken at %s MHz under the power cap)"
-                                  % (peaks["source"], "%.0f" % sm if sm is not None else "unsampled",
-                                     peaks.get("sustained_sm_mhz")))
+    burst, sust = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    if sm is None or not smax or sm >= smax:
+        return burst, ("%s bf16 dense, burst (this run's median SM clock %s MHz is the maximum; the sustained "
+                       "figure was taken at %s MHz under the power cap)"
+                       % (peaks["source"], "%.0f" % sm if sm is not None else "unsampled",
+                          peaks.get("sustained_sm_mhz")))
+    scaled = burst * sm / smax
+    if scaled >= sust:
+        return scaled, ("%s bf16 dense, burst %.0f TFLOP/s scaled by this run's median SM clock %.0f MHz over the "
+                        "maximum %.0f MHz (the sustained figure, %.0f at %s MHz, is the floor)"
+                        % (peaks["source"], burst, sm, smax, sust, peaks.get("sustained_sm_mhz")))
+    return sust, ("%s bf16 dense, sustained (this run's median SM clock %.0f MHz; the burst figure scaled to it, "
+                  "%.0f TFLOP/s, is below the sustained floor)" % (peaks["source"], sm, scaled))
 
 
 def attention_traffic():

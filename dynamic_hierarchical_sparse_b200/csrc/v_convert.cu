@@ -25,16 +25,29 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, bool& bad) {
 
 __global__ void __launch_bounds__(kConvThreads)
     v_to_f16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16, long long nvec, uint32_t* status) {
+  // kUnroll independent 16-byte loads in flight per thread before any store
+  constexpr int kUnroll = 4;
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(kConvThreads) + threadIdx.x; i < nvec;
-       i += static_cast<long long>(gridDim.x) * kConvThreads) {
-    const uint4 x = __ldcs(v + i);
-    uint4 y;
-    y.x = bf16x2_to_f16x2(x.x, bad);
-    y.y = bf16x2_to_f16x2(x.y, bad);
-    y.z = bf16x2_to_f16x2(x.z, bad);
-    y.w = bf16x2_to_f16x2(x.w, bad);
-    v16[i] = y;
+  const long long stride = static_cast<long long>(gridDim.x) * kConvThreads;
+  for (long long i0 = blockIdx.x * static_cast<long long>(kConvThreads) + threadIdx.x; i0 < nvec;
+       i0 += kUnroll * stride) {
+    uint4 x[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = i0 + u * stride;
+      x[u] = i < nvec ? __ldcs(v + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = i0 + u * stride;
+      if (i >= nvec) break;
+      uint4 y;
+      y.x = bf16x2_to_f16x2(x[u].x, bad);
+      y.y = bf16x2_to_f16x2(x[u].y, bad);
+      y.z = bf16x2_to_f16x2(x[u].z, bad);
+      y.w = bf16x2_to_f16x2(x[u].w, bad);
+      v16[i] = y;
+    }
   }
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(status, kDevCheck);
 }
@@ -48,7 +61,7 @@ cudaError_t launch_v_to_f16(const void* v, void* v16, long long n, uint32_t* sta
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const long long nvec = n / 8;
-  const long long need = (nvec + kConvThreads - 1) / kConvThreads;
+  const long long need = (nvec + 4LL * kConvThreads - 1) / (4LL * kConvThreads);  // four vectors per thread
   const int grid = static_cast<int>(need < 8LL * sms ? need : 8LL * sms);
   v_to_f16_kernel<<<grid, kConvThreads, 0, stream>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), nvec,
                                                      status);

@@ -417,3 +417,17 @@ def test_segment_rejects_before_launch(case):
                              P(256), 255, P(0))
         want = 3
     assert got == want
+
+
+def test_tensor_peak_follows_the_sampled_clock():
+    """The roofline's bf16 denominator: the burst GEMM figure at the maximum
+    clock, scaled with the run's median SM clock below it, never under the
+    sustained figure."""
+    import bench
+
+    pk = {"bf16_tflops": 1630.0, "bf16_tflops_sustained": 1374.2, "sustained_sm_mhz": 1237.0,
+          "sm_max_mhz": 1965.0, "source": "measured"}
+    assert bench.tensor_peak(pk, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})[0] == 1630.0
+    assert bench.tensor_peak(pk, {"sm_mhz": None})[0] == 1630.0
+    assert abs(bench.tensor_peak(pk, {"sm_mhz": 1848.5, "sm_max_mhz": 1965.0})[0] - 1630.0 * 1848.5 / 1965.0) < 1e-9
+    assert bench.tensor_peak(pk, {"sm_mhz": 1237.0, "sm_max_mhz": 1965.0})[0] == 1374.2
