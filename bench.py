@@ -670,7 +670,8 @@ def bench_segment_micro(args):
     """Online chunking alone on the 128K LLaMA key shape (K [131072, 8, 128]
     bf16, 268 MB), keys with planted segments U[256, 1024] (the 128K
     workload's chunk lengths), rule threshold 0.5, min 256, max 1024.  One call
-    is three launches (adjacent-key similarity bits, the walk, compaction).
+    is two launches (adjacent-key similarity bits, then the walk, which writes the chunk
+    bounds itself for a batch of one sequence).
     Algorithmic bytes: every key read once plus the two bitmaps written and
     read (T/8 bytes each way) and the bounds written."""
     from dynamic_hierarchical_sparse_b200 import api
@@ -716,11 +717,11 @@ def bench_segment_micro(args):
                    "rule": {"threshold": cfg["rule"].threshold, "min_len": cfg["rule"].min_len,
                             "max_len": cfg["rule"].max_len},
                    "num_chunks": n, "l2": "no flush: keys %.2f GB > 126 MB L2" % (key_bytes / 1e9)},
-        "roofline": {"kernel": "dhsa_segment (3 launches; adjacent_sim_kernel dominant)", "bound": "hbm",
+        "roofline": {"kernel": "dhsa_segment (2 launches; adjacent_sim_kernel dominant)", "bound": "hbm",
                      "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "peak_kind": "%s copy bandwidth" % peaks["source"],
                      "note": "whole call timed: the walk and compaction count against it"},
-        "gpu_launches": 3 * args.steps,  # similarity, walk, compaction per call
+        "gpu_launches": 2 * args.steps,  # similarity, walk (with the compaction: one sequence) per call
         "clocks": clk,
     }
     if not args.no_cpu_baseline:
@@ -801,7 +802,7 @@ def bench_online_chunking(args):
                    "rule": {"threshold": rule.threshold, "min_len": rule.min_len, "max_len": rule.max_len},
                    "num_chunks": int(hb.shape[0] - 1), "budget": _budget_str(inp.budget)},
         "ms_segment_and_readback": part[0], "ms_plan": part[1], "ms_attention": part[2],
-        "gpu_launches": 8 * args.steps,  # segment 3, plan 3, f16 copy of V 1, attention 1 per step
+        "gpu_launches": 7 * args.steps,  # segment 2 (one sequence), plan 3, f16 copy of V 1, attention 1 per step
         "clocks": clk,
     }), flush=True)
 

@@ -31,7 +31,8 @@
 //     step by one thread instead.  Chunk starts are set in a second bitmap.
 //  3. segment_compact_kernel: one CTA turns the start bitmap into chunk_bounds
 //     (a block-wide scan of per-thread bit counts), then seq_chunk_ptr by binary
-//     search of each sequence's first token.
+//     search of each sequence's first token.  A batch of one sequence skips this
+//     launch: its walk CTA, which holds every start, writes the bounds itself.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -248,7 +249,9 @@ __device__ __forceinline__ void set_start(uint32_t* start_bits, int p) {
 
 __global__ void __launch_bounds__(kWalkThreads)
     segment_walk_kernel(const uint32_t* __restrict__ drop, const int* __restrict__ cu_seqlens, int min_len,
-                        int max_len, uint32_t* __restrict__ start_bits, uint32_t* status) {
+                        int max_len, uint32_t* __restrict__ start_bits, uint32_t* status, int compact,
+                        int* __restrict__ chunk_bounds, long long capacity, int* __restrict__ seq_chunk_ptr,
+                        int* __restrict__ num_chunks) {
   extern __shared__ __align__(128) unsigned char walk_smem_raw[];
   WalkSmem& S = *reinterpret_cast<WalkSmem*>(walk_smem_raw);
   __shared__ __align__(8) uint64_t bar;
@@ -469,6 +472,48 @@ __global__ void __launch_bounds__(kWalkThreads)
     __syncthreads();  // s_b, s_done and the start list are rewritten by the next round
     if (fin) break;
   }
+  if (!compact) return;
+  // A batch of one sequence: the start bitmap -> chunk_bounds here, without
+  // the compaction launch (every start is set, and the block's atomics are
+  // visible to it after the barrier).  An exclusive prefix of the threads'
+  // start counts over runs of consecutive words.
+  __syncthreads();
+  const int nw = (s1 + 31) >> 5;
+  const int per = (nw + kWalkThreads - 1) / kWalkThreads;
+  const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(start_bits[w]);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) S.warp_cnt[warp] = incl;
+  __syncthreads();
+  long long pos = incl - cnt;
+  int total = 0;
+  for (int w = 0; w < kWalkThreads / 32; ++w) {
+    if (w < warp) pos += S.warp_cnt[w];
+    total += S.warp_cnt[w];
+  }
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = start_bits[w];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < capacity) chunk_bounds[pos] = (w << 5) + bit;
+      ++pos;
+    }
+  }
+  if (tid == 0) {
+    if (total > capacity) report(status, kDevCheck);
+    const int n = static_cast<int>(min(static_cast<long long>(total), capacity));
+    chunk_bounds[n] = s1;
+    *num_chunks = total;
+    seq_chunk_ptr[0] = 0;
+    seq_chunk_ptr[1] = n;
+  }
 }
 
 __global__ void __launch_bounds__(kCompactThreads)
@@ -567,10 +612,14 @@ cudaError_t launch_segment(const void* k, int dtype, int total_tokens, int num_k
       constexpr int walk_smem = static_cast<int>(sizeof(WalkSmem));
       e = cudaFuncSetAttribute(segment_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, walk_smem);
       if (e != cudaSuccess) return e;
+      // one sequence: the walk writes the chunk bounds itself
+      const int compact = num_seqs == 1 ? 1 : 0;
       segment_walk_kernel<<<num_seqs, kWalkThreads, walk_smem, stream>>>(drop, cu_seqlens, min_len, max_len,
-                                                                         start_bits, status);
+                                                                         start_bits, status, compact,
+                                                                         chunk_bounds, capacity, seq_chunk_ptr,
+                                                                         num_chunks);
       e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
+      if (e != cudaSuccess || compact) return e;
     }
   }
   segment_compact_kernel<<<1, kCompactThreads, 0, stream>>>(start_bits, total_tokens, cu_seqlens, num_seqs,
