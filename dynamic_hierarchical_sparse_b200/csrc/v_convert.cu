@@ -2,8 +2,8 @@
 // O += P V, with P in f16 (tcgen05.mma kind::f16 takes A and B of one type).
 // bf16 -> f16 is exact for magnitudes up to 65504 (f16 has the more
 // significant bits; below 2^-14 it goes subnormal, an absolute error of at
-// most 2^-25).  Larger magnitudes, and NaN, have no f16 counterpart here: they
-// are reported (kDevCheck) and written saturated.
+// most 2^-25).  Larger magnitudes and NaN are reported (kDevCheck): a larger
+// magnitude is written saturated to +-65504, a NaN as a NaN.
 //
 // HBM-bound: 2 bytes read and 2 written per element, 16-byte vectors,
 // grid-stride over a grid of whole waves.
