@@ -162,6 +162,11 @@ DHSA_API dhsa_status dhsa_topk_select(const float* scores, const dhsa_problem* p
                              void* stream);
 
 /* ---- steps 1-3 ------------------------------------------------------------
+ * dhsa_chunk_reduce, dhsa_chunk_similarity and dhsa_topk_select in one call,
+ * from q and k to the plan (On-Device page, Abstract: chunk representations,
+ * chunk-level similarity, upsampled scores deciding the kept interactions;
+ * Memory-Constrained page, abstract: importance estimated per chunk and
+ * carried to the token pairs, causal dependencies kept).
  * Workspace: dhsa_plan_workspace_size bytes, 256-byte aligned, device.  It
  * holds the status word, qc, kc and the score matrix (and, for a per-KV-head
  * plan, the summed query chunks [Hkv, n, d] fp32; the score matrix is then
@@ -306,11 +311,12 @@ DHSA_API dhsa_status dhsa_segment(const void* k, int32_t dtype, int32_t num_kv_h
                                   size_t workspace_bytes, void* stream);
 
 /* ---- steps 1-3 without a caller workspace ----------------------------------
- * No counterpart in the paper: an interface addition for callers that cannot
- * allocate device memory at the point where they plan, such as code that runs
- * inside another framework's allocator-free region, a plugin that is handed
- * only its input and output buffers, or a process whose allocations go through
- * a pool it does not own.  Same inputs, outputs and results as dhsa_plan; the
+ * The computation is dhsa_plan's (On-Device page, Abstract; steps 1-3 above).
+ * The pages have no counterpart of this entry point: an interface addition
+ * for callers that cannot allocate device memory at the point where they plan,
+ * such as code that runs inside another framework's allocator-free region, a
+ * plugin that is handed only its input and output buffers, or a process whose
+ * allocations go through a pool it does not own.  Same inputs, outputs and results as dhsa_plan; the
  * scratch (status word, qc, kc, score matrix) lives in one fixed device array
  * inside the library, DHSA_PLAN_NOALLOC_MAX_SCRATCH bytes per device, which
  * every GPU that loads the library holds until the process exits.
