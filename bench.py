@@ -47,7 +47,7 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # any other source reports traffic as null.
 ATTN_TRAFFIC_CAPTURE = {
     "bytes": 10.466e9,  # 9.427 GB read + 1.040 GB written
-    "source_sha256": "5e739af4ab8cc692fea69f54f4e1d2c3212a34bfc245f3bb1b1182e4f61a703e",
+    "source_sha256": "63ac24714324faddb9475e89fc9fbdd1d3220fd58ea2549a9a07e11adb16c24b",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:attention_pair -s 1 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-micro"),
 }

@@ -87,7 +87,7 @@ constexpr int kVStages = 3;     // V ring depth (K uses 2)
 // O is rescaled whenever a warp's running max grows (threshold 0 in log2
 // units): the row's largest weight is then exp2(0) = 1, exact.  A lazy
 // threshold (2^8) let the running max lag, so the largest weight was rounded
-// (to bf16 then, 2^-9 relative) and that rounding reached O directly: 0.026 of error
+// (to bf16 then, up to 2^-8 relative) and that rounding reached O directly: 0.026 of error
 // at |O| = 4.4 at 128K, against 0.017 with every growth rescaled, for about
 // 4 % of attention time.
 constexpr float kRescaleLog2 = 0.0f;
@@ -211,10 +211,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// P as an f16 pair: the weights lie in [0, 1], where f16 keeps 11 significant
-// bits against bf16's 8, so rounding them perturbs O by at most 2^-12 max|V|
-// (2^-9 max|V| in bf16, which at |O| in [4, 8) adds to the output's own
-// rounding of up to 2^-6 and can pass a 2e-2 error bound).
+// P as an f16 pair: f16 keeps 11 significant bits against bf16's 8, so each
+// weight rounds by at most 2^-11 of itself and the weights' rounding moves O
+// by at most 2^-11 max|V| (2^-8 max|V| in bf16, which at |O| in [4, 8) adds
+// to the output's own rounding of up to 2^-6 and can pass a 2e-2 bound).
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -12,10 +12,11 @@ TIE_REL = 1e-5      # near-tie rule on the oracle's k-th / (k+1)-th scores
 ATOL_BF16 = 2e-2    # max-abs gate on bf16 outputs
 ATOL_F32 = 1e-4     # max-abs gate on fp32 outputs
 # Relative Frobenius gates, beside the absolute ones.  bf16: the kernel adds
-# two roundings to the exact computation, the bf16 output (2^-9 relative at
-# most, 2^-9/sqrt(3) RMS) and the bf16 attention weights P before the PV
-# product (the same per weight, independent across keys), about 0.2 % RMS
-# together; 1e-2 leaves five times that.  The ratio does not depend on the
+# two roundings to the exact computation, the bf16 output (2^-8 relative at
+# most, the unit roundoff of an 8-bit significand; about 0.17 % RMS) and the
+# 16-bit attention weights P before the PV product (bf16 when this gate was
+# set, the same per weight and independent across keys; f16 now, 2^-11 at
+# most), about 0.2 % RMS together; 1e-2 leaves about five times that.  The ratio does not depend on the
 # output's scale, so it binds on diffuse rows (N(0,1) inputs, |O| ~ 0.02)
 # where a 2e-2 absolute gate alone would allow a 100 % error.  fp32: the FFMA
 # kernel's error is ~1e-6 relative; 1e-4 is the absolute gate's own figure.
