@@ -126,7 +126,15 @@ def kept_pairs(bounds, row_ptr, col, num_chunks):
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs.
+
+    nvidia-smi starts sampling before the timed region (it needs a moment to
+    start), so each line is stamped with the host time it arrived, and only the
+    lines that arrived between mark_start() and mark_stop() count.  If none did
+    (output held back by buffering, or a region shorter than one interval), all
+    lines are used and the record says so."""
+
+    INTERVAL_MS = 100
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -135,14 +143,16 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (host time of arrival, line)
         self.thread = None
+        self.t0 = None
+        self.t1 = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -152,7 +162,15 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        """Host time at which the timed region starts (call just before it)."""
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        """Host time at which the timed region has ended (call after the synchronize)."""
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
@@ -164,22 +182,31 @@ class ClockSampler:
             self.proc.kill()
         if self.thread is not None:
             self.thread.join(timeout=5)
-        sm, smax, reasons = [], None, set()
+        return self.summarise(self.lines, self.t0, self.t1)
+
+    @staticmethod
+    def summarise(lines, t0, t1):
+        """Median SM clock, maximum clock and throttle reasons of the samples
+        that arrived in [t0, t1], else of all samples."""
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        rows = []  # (arrival, sm MHz, max MHz, active reasons)
+        for t, ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                sm, smax = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            rows.append((t, sm, smax, {nm for nm, val in zip(names, parts[5:9]) if val.lower().startswith("active")}))
+        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        use = inside if inside else rows
+        reasons = set().union(*(r[3] for r in use)) if use else set()
+        return {"sm_mhz": statistics.median(r[1] for r in use) if use else None,
+                "sm_max_mhz": use[-1][2] if use else None,
+                "reasons": sorted(reasons), "samples": len(use), "samples_total": len(rows),
+                "window": "samples that arrived during the timed region" if inside else
+                          "all samples (none arrived during the timed region)"}
 
 
 def _dist_setup(n_gpus: int):
@@ -449,6 +476,7 @@ def bench_gpu(args):
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
+    clocks.mark_start()
     start.record(stream)
     for i in range(args.steps):
         if flush is not None:
@@ -460,6 +488,7 @@ def bench_gpu(args):
         ev[i][2].record(stream)
     stop.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_stop()
     clk = clocks.stop()
     _barrier(world)
     elapsed_s = start.elapsed_time(stop) / 1e3
@@ -696,11 +725,13 @@ def bench_segment_micro(args):
     clocks = ClockSampler(0)
     clocks.start()
     time.sleep(0.3)
+    clocks.mark_start()
     e0.record(stream)
     for _ in range(args.steps):
         seg(k)
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_stop()
     clk = clocks.stop()
     t = e0.elapsed_time(e1) / 1e3 / args.steps
     T = cfg["tokens"]
@@ -787,9 +818,11 @@ def bench_online_chunking(args):
     clocks.start()
     time.sleep(0.3)
     torch.cuda.synchronize()
+    clocks.mark_start()
     for i in range(args.steps):
         step(evs[i])
     torch.cuda.synchronize()
+    clocks.mark_stop()
     clk = clocks.stop()
     total = sum(e[0].elapsed_time(e[3]) for e in evs) / 1e3
     part = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
