@@ -73,26 +73,25 @@ def _peaks():
 
 def tensor_peak(peaks, clk):
     """The bf16 peak a kernel timed in this run is held against, from the SM
-    clock sampled during the timed region: the burst figure (a GEMM timed
-    alone at the maximum clock) scaled by this run's median clock over the
-    maximum, since tensor throughput follows the clock, and never below the
-    sustained figure (a seconds-long loop under the power cap, at its lower
-    clock).  At the maximum clock this is the burst figure itself.  Returns
-    (peak, kind)."""
+    clock sampled during the timed region.  Two GEMM figures were measured:
+    the burst one (timed alone, taken at the maximum clock) and the sustained
+    one (a seconds-long loop under the power cap, at its recorded median
+    clock).  The peak is the straight line through those two (clock, TFLOP/s)
+    points at this run's median clock, kept between the two figures: the burst
+    figure at the maximum clock, the sustained one at or below its clock.  A
+    run whose clock was not sampled gets the burst figure.  Returns (peak, kind)."""
     sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz") or peaks.get("sm_max_mhz")
-    burst, sust = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
-    if sm is None or not smax or sm >= smax:
-        return burst, ("%s bf16 dense, burst (this run's median SM clock %s MHz is the maximum; the sustained "
-                       "figure was taken at %s MHz under the power cap)"
-                       % (peaks["source"], "%.0f" % sm if sm is not None else "unsampled",
-                          peaks.get("sustained_sm_mhz")))
-    scaled = burst * sm / smax
-    if scaled >= sust:
-        return scaled, ("%s bf16 dense, burst %.0f TFLOP/s scaled by this run's median SM clock %.0f MHz over the "
-                        "maximum %.0f MHz (the sustained figure, %.0f at %s MHz, is the floor)"
-                        % (peaks["source"], burst, sm, smax, sust, peaks.get("sustained_sm_mhz")))
-    return sust, ("%s bf16 dense, sustained (this run's median SM clock %.0f MHz; the burst figure scaled to it, "
-                  "%.0f TFLOP/s, is below the sustained floor)" % (peaks["source"], sm, scaled))
+    burst, sust, s_mhz = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"], peaks.get("sustained_sm_mhz")
+    if sm is None or not smax or sm >= smax or not s_mhz or s_mhz >= smax:
+        return burst, ("%s bf16 dense, burst (this run's median SM clock %s MHz, the maximum %s MHz)"
+                       % (peaks["source"], "%.0f" % sm if sm is not None else "unsampled", smax))
+    if sm <= s_mhz:
+        return sust, ("%s bf16 dense, sustained (this run's median SM clock %.0f MHz is at or below the %.0f MHz "
+                      "of the sustained figure)" % (peaks["source"], sm, s_mhz))
+    peak = sust + (burst - sust) * (sm - s_mhz) / (smax - s_mhz)
+    return peak, ("%s bf16 dense at this run's median SM clock %.0f MHz: the line through the sustained figure "
+                  "(%.0f TFLOP/s at %.0f MHz) and the burst figure (%.0f at the maximum %.0f MHz)"
+                  % (peaks["source"], sm, sust, s_mhz, burst, smax))
 
 
 def attention_traffic():
@@ -582,6 +581,7 @@ def bench_gpu(args):
         "roofline": {
             "kernel": kernel, "bound": bound, "achieved": achieved_tflops,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved_tflops / peak, "peak_kind": peak_kind,
+            "frac_of_burst": (achieved_tflops / peaks["bf16_tflops"]) if bound == "tensor" else None,
             "frac_of_sustained": (achieved_tflops / peaks["bf16_tflops_sustained"]) if bound == "tensor" else None,
             "traffic": traffic, "traffic_kind": traffic_kind,
             "algorithmic_flops_per_launch": flops_attn,

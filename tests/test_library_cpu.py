@@ -420,14 +420,20 @@ def test_segment_rejects_before_launch(case):
 
 
 def test_tensor_peak_follows_the_sampled_clock():
-    """The roofline's bf16 denominator: the burst GEMM figure at the maximum
-    clock, scaled with the run's median SM clock below it, never under the
-    sustained figure."""
+    """The roofline's bf16 denominator: the straight line through the two
+    measured GEMM figures (sustained at its median clock, burst at the
+    maximum), at the run's median SM clock, kept between the two."""
     import bench
 
     pk = {"bf16_tflops": 1630.0, "bf16_tflops_sustained": 1374.2, "sustained_sm_mhz": 1237.0,
           "sm_max_mhz": 1965.0, "source": "measured"}
     assert bench.tensor_peak(pk, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})[0] == 1630.0
     assert bench.tensor_peak(pk, {"sm_mhz": None})[0] == 1630.0
-    assert abs(bench.tensor_peak(pk, {"sm_mhz": 1848.5, "sm_max_mhz": 1965.0})[0] - 1630.0 * 1848.5 / 1965.0) < 1e-9
     assert bench.tensor_peak(pk, {"sm_mhz": 1237.0, "sm_max_mhz": 1965.0})[0] == 1374.2
+    assert bench.tensor_peak(pk, {"sm_mhz": 1100.0, "sm_max_mhz": 1965.0})[0] == 1374.2
+    mid = bench.tensor_peak(pk, {"sm_mhz": (1237.0 + 1965.0) / 2, "sm_max_mhz": 1965.0})[0]
+    assert abs(mid - (1374.2 + 1630.0) / 2) < 1e-9
+    # the loaded clock of a 128K bench run: 1702 MHz -> 1537.7 TFLOP/s, above the burst figure
+    # scaled through the origin (1411.8), which the sustained point shows to be too low
+    p1702 = bench.tensor_peak(pk, {"sm_mhz": 1702.0, "sm_max_mhz": 1965.0})[0]
+    assert abs(p1702 - (1374.2 + 255.8 * 465.0 / 728.0)) < 1e-9 and p1702 > 1630.0 * 1702.0 / 1965.0
