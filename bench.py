@@ -47,7 +47,7 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # any other source reports traffic as null.
 ATTN_TRAFFIC_CAPTURE = {
     "bytes": 10.466e9,  # 9.427 GB read + 1.040 GB written
-    "source_sha256": "63ac24714324faddb9475e89fc9fbdd1d3220fd58ea2549a9a07e11adb16c24b",
+    "source_sha256": "1bb96dae4a6fed858207fa584db122048db77d57264dbcc20e44acadc74ae586",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:attention_pair -s 1 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-micro"),
 }

@@ -211,10 +211,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// P as an f16 pair: f16 keeps 11 significant bits against bf16's 8, so each
-// weight rounds by at most 2^-11 of itself and the weights' rounding moves O
-// by at most 2^-11 max|V| (2^-8 max|V| in bf16, which at |O| in [4, 8) adds
-// to the output's own rounding of up to 2^-6 and can pass a 2e-2 bound).
+// P as an f16 pair: 11 significant bits against bf16's 8.  A weight rounds by
+// at most 2^-11 of itself (by up to 2^-25 below 2^-14, where f16 is subnormal),
+// so O moves by at most 2^-11 max|V|, plus 2^-25 max|V| / l per subnormal weight;
+// in bf16 by 2^-8 max|V|, which with the output's own 2^-6 can pass a 2e-2 bound.
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -190,7 +190,9 @@ DHSA_API dhsa_status dhsa_plan(const void* q, const void* k, const dhsa_problem*
  * each call, then (bf16 problems) an f16 copy of v, T*Hkv*d*2 bytes, written by
  * each call: the tensor cores take the softmax weights P and V in f16 (11
  * significant bits against bf16's 8: each weight rounds by at most 2^-11 of
- * itself, so the weights' rounding moves out by at most 2^-11 max|v|).  A |v| above 65504 or a NaN is reported as
+ * itself, or by up to 2^-25 below 2^-14 where f16 is subnormal, so out moves
+ * by at most 2^-11 max|v| plus 2^-25 max|v| / l per weight below 2^-14, l the
+ * row's sum of weights).  A |v| above 65504 or a NaN is reported as
  * DHSA_ERR_DEVICE_CHECK through dhsa_workspace_status (the copy holds +-65504
  * for the former, NaN for the latter).
  * A workspace serves one call at a time: calls that may overlap on the GPU
