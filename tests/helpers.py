@@ -46,8 +46,9 @@ def compare_plans(rows_gpu, ref, inp, budget):
     best admissible scores are within TIE_REL of the larger of |s_k|, |s_k+1|
     and the row's largest |score| (fp32 score error scales with the row, not
     with one score); even then the GPU row must
-    be a valid selection whose members all score within that margin of the
-    threshold.  Returns the list of tolerated near-tie rows.
+    be a valid selection: its members all score at least the threshold less
+    that margin, and it holds every candidate that scores more than the
+    threshold plus the margin.  Returns the list of tolerated near-tie rows.
     """
     rows_ref = O.plan_rows(ref["row_ptr"], ref["col"])
     assert len(rows_gpu) == len(rows_ref)
@@ -70,6 +71,9 @@ def compare_plans(rows_gpu, ref, inp, budget):
         S = ref["S"][h, i]
         for j in g[:-1]:
             assert S[j] >= sk - margin, (r, j)
+        # and every candidate clearly above the threshold is kept
+        clear = [j for j in range(int(ptr[b]), i) if S[j] > sk + margin]
+        assert set(clear) <= set(g), ("a candidate clearly above the threshold is missing", r, g, clear)
         tolerated.append(r)
     return tolerated
 
