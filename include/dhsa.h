@@ -38,7 +38,8 @@
  *   DHSA_ERR_CUDA.  Errors found by the kernels themselves (a bounded wait that
  *   ran out, an index check) are written to a status word at the start of the
  *   workspace and read with dhsa_workspace_status.
- * - No C++ exception crosses this interface.  All entry points are reentrant.
+ * - No C++ exception crosses this interface.  All entry points are reentrant,
+ *   except that calls of dhsa_plan_noalloc share one device array (see there).
  */
 #ifndef DHSA_H_
 #define DHSA_H_
@@ -152,7 +153,8 @@ DHSA_API dhsa_status dhsa_chunk_similarity(const float* qc, const float* kc,
  * lower j), plus the diagonal i.  Because every token pair of chunks (i, j)
  * inherits score(i, j), this is the token-level keep set of the pages'
  * upsampling step, stored per chunk.
- *   row_ptr  device int32 [Hq*n + 1]  (CSR offsets, written)
+ *   row_ptr  device int32 [rows + 1]  (CSR offsets, written; rows = Hq*n, or
+ *                                      Hkv*n for a per-KV-head plan)
  *   col      device int32 [nnz]       (ascending chunk ids; the diagonal is
  *                                      the last entry of its row)
  *   nnz      must equal dhsa_plan_nnz() for the same problem and budget. */
