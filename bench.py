@@ -47,7 +47,7 @@ DEFAULT_WORKLOAD = W.LLAMA_128K.name
 # any other source reports traffic as null.
 ATTN_TRAFFIC_CAPTURE = {
     "bytes": 10.466e9,  # 9.427 GB read + 1.040 GB written
-    "source_sha256": "1bb96dae4a6fed858207fa584db122048db77d57264dbcc20e44acadc74ae586",
+    "source_sha256": "14d72c73ae0e794dede9b6cad0ccff10c01b6bb6c5dd53e49fd3ff01f4e94cbd",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:attention_pair -s 1 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-micro"),
 }
