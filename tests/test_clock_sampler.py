@@ -10,10 +10,9 @@ import time
 import bench
 
 FAKE_SMI = """#!{python}
-import sys, time
-t0 = time.time()
+import os, sys, time
 while True:
-    busy = time.time() - t0 >= {idle_s}
+    busy = os.path.exists({flag!r})
     sys.stdout.write("0, %d, 1965, 500.00, 0x0, Not Active, Not Active, Not Active, %s\\n"
                      % (1700 if busy else 1965, "Active" if busy else "Not Active"))
     sys.stdout.flush()
@@ -21,18 +20,23 @@ while True:
 """
 
 
-def _install_fake_smi(tmp_path, monkeypatch, idle_s):
+def _install_fake_smi(tmp_path, monkeypatch, flag):
     path = tmp_path / "nvidia-smi"
-    path.write_text(FAKE_SMI.format(python=sys.executable, idle_s=idle_s))
+    path.write_text(FAKE_SMI.format(python=sys.executable, flag=str(flag)))
     path.chmod(path.stat().st_mode | stat.S_IXUSR)
     monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ.get("PATH", ""))
 
 
 def test_median_and_reasons_come_from_the_timed_region(tmp_path, monkeypatch):
-    _install_fake_smi(tmp_path, monkeypatch, idle_s=0.4)
+    flag = tmp_path / "busy"
+    _install_fake_smi(tmp_path, monkeypatch, flag)
     clocks = bench.ClockSampler(0)
     clocks.start()
-    time.sleep(0.6)  # the stand-in reports idle clocks for its first 0.4 s
+    deadline = time.time() + 30
+    while len(clocks.lines) < 10 and time.time() < deadline:  # idle samples before the region
+        time.sleep(0.02)
+    flag.touch()  # the stand-in reports loaded clocks from here on
+    time.sleep(0.1)
     clocks.mark_start()
     time.sleep(0.3)
     clocks.mark_stop()
